@@ -1,0 +1,110 @@
+"""Seeded synthetic inputs shared by the tests, the bench and the oracle checks.
+
+This module holds no attention arithmetic: it only draws random tensors and
+picks row samples.  Both the CUDA path and the oracle are fed from here.
+
+Recipe: a CPU ``torch.Generator`` seeded with ``seed`` draws Q, K, V in that
+order with ``torch.randn(B, H, N, d)`` in float32; Q is multiplied by
+``q_std``; all three are rounded to bfloat16 (round to nearest even).  The
+oracle reads the bfloat16 values, widened exactly.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    """One attention-forward problem: shapes, mask, scale and input seed."""
+
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool
+    seed: int
+    q_std: float = 1.0
+    sample_rows: int = 0  # 0 = every row is checked against the oracle
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def flops(self) -> float:
+        """4*B*H*N^2*d, halved for causal (the counting convention)."""
+        f = 4.0 * self.B * self.H * self.N * self.N * self.d
+        return f / 2 if self.causal else f
+
+    def as_config(self) -> dict:
+        return {
+            "workload": self.name, "B": self.B, "H": self.H, "N": self.N,
+            "d": self.d, "causal": self.causal, "seed": self.seed,
+            "q_std": self.q_std, "scale": self.scale,
+        }
+
+
+# The five problems of the benchmark plan, named by their shape.
+WORKLOADS = {
+    w.name: w
+    for w in (
+        Workload("b1h1n256d64", 1, 1, 256, 64, False, 0),
+        Workload("b4h16n4096d64", 4, 16, 4096, 64, False, 1, sample_rows=4096),
+        Workload("b2h16n8192d128_causal", 2, 16, 8192, 128, True, 2, sample_rows=4096),
+        Workload("b1h32n32768d128_causal_q4", 1, 32, 32768, 128, True, 3, q_std=4.0,
+                 sample_rows=2048),
+        Workload("b1h8n131072d128_causal", 1, 8, 131072, 128, True, 4, sample_rows=1024),
+    )
+}
+
+
+def make_qkv(B: int, H: int, N: int, d: int, seed: int, q_std: float = 1.0,
+             k_std: float = 1.0, v_std: float = 1.0):
+    """Q, K, V as contiguous CPU bfloat16 tensors [B, H, N, d]."""
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    shape = (B, H, N, d)
+    q = torch.randn(shape, generator=g, dtype=torch.float32)
+    k = torch.randn(shape, generator=g, dtype=torch.float32)
+    v = torch.randn(shape, generator=g, dtype=torch.float32)
+    if q_std != 1.0:
+        q.mul_(q_std)
+    if k_std != 1.0:
+        k.mul_(k_std)
+    if v_std != 1.0:
+        v.mul_(v_std)
+    return (q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16))
+
+
+def make_workload_inputs(w: Workload):
+    return make_qkv(w.B, w.H, w.N, w.d, w.seed, w.q_std)
+
+
+def sample_rows(B: int, H: int, N: int, count: int, seed: int) -> torch.Tensor:
+    """Rows (b, h, i) to check: ``count`` random ones plus forced edge rows.
+
+    The random rows come from ``torch.randperm`` with generator seed
+    1000 + seed; the forced rows are i in {0, 1, 127, 128, N-1} (those that
+    exist) for h in {0, H-1}, b in {0, B-1}.  ``count <= 0`` returns every row.
+    """
+    total = B * H * N
+    if count <= 0 or count >= total:
+        idx = torch.arange(total)
+    else:
+        g = torch.Generator(device="cpu").manual_seed(1000 + int(seed))
+        idx = torch.randperm(total, generator=g)[:count]
+        forced = []
+        for b in sorted({0, B - 1}):
+            for h in sorted({0, H - 1}):
+                for i in (0, 1, 127, 128, N - 1):
+                    if 0 <= i < N:
+                        forced.append((b * H + h) * N + i)
+        idx = torch.unique(torch.cat([idx, torch.tensor(forced, dtype=torch.long)]))
+    b = idx // (H * N)
+    h = (idx // N) % H
+    i = idx % N
+    return torch.stack([b, h, i], dim=1)
