@@ -1,0 +1,610 @@
+// Fused exact softmax attention forward for B200 (sm_100a), and the C ABI
+// declared in include/fa.h.
+//
+// What it computes: O = softmax(scale * Q K^T [+ causal mask]) V and the
+// row log-sum-exp (lihaoran.work "FlashAttention: the intermediate matrix
+// comes first", the opening formula).  How: the online block update of
+// liminalml.com "FlashAttention" -- per query row a running maximum m,
+// denominator l and unnormalised numerator u; a tile whose scores raise the
+// maximum rescales u and l by e^(m - m') before its own terms are added
+// (the 5 -> 10 question on the same page), and the output is u / l after the
+// last tile.  Scores and probabilities live only in tensor memory; the N x N
+// matrix never reaches HBM (sadullah.online "Flash Attention Explained",
+// fused tiled computation; interactiveml.org "FlashAttention saves the
+// matrix, not the quadratic work").
+//
+// CTA layout (384 threads, one CTA per SM):
+//   warp 0      TMA producer: Q tiles once, then K/V tiles through a ring of
+//               shared-memory stages guarded by full/empty mbarriers.
+//   warp 1      TMEM owner and MMA issuer (one thread): S_t = Q_t K^T
+//               (SS MMA, M=128 N=128 K=d) and O_t += P_t V (TS MMA, P from
+//               TMEM, M=128 N=d K=128), completion signalled by tcgen05.commit.
+//   warps 2-3   idle.
+//   warps 4-7   softmax + epilogue for query tile 0 (one thread per row).
+//   warps 8-11  softmax + epilogue for query tile 1.
+// Each CTA owns 2 query tiles of 128 rows (256 rows of one head) so that the
+// softmax of one tile overlaps the MMAs of the other.
+//
+// Tensor memory (512 columns x 128 lanes of 32 bit):
+//   [0,128)      S_0, fp32; P_0 (bf16 pairs) overwrites its first 64 columns
+//   [128,256)    S_1 / P_1
+//   [256,256+d)  O_0 accumulator, fp32
+//   [256+d, 256+2d) O_1 accumulator
+//
+// Softmax runs in base 2 with log2(e) folded into the scale: x = s * scale *
+// log2 e, p = 2^(x - m).  The reference maximum m is only raised when a tile
+// exceeds it by more than 8 (a factor 256), so most tiles skip the O rescale;
+// p <= 256 stays exact enough in bf16 and the final u / l uses the same m,
+// so the result is unchanged.
+//
+// Every wait is bounded: a wait that runs out sets an abort flag in shared
+// memory and a bit in the device status word; all roles then unwind, copies
+// in flight are drained, and TMEM is released.  Nothing traps.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "sm100.cuh"
+
+namespace fa {
+
+constexpr int kBM = 128;       // query rows per tile
+constexpr int kBN = 128;       // keys per tile
+constexpr int kQTiles = 2;     // query tiles per CTA
+constexpr int kThreads = 384;  // 12 warps
+constexpr int kSoftmaxWarp0 = 4;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr uint32_t kTmemCols = 512;
+constexpr int kChunkBytes = kBM * 64 * 2;  // one 64-wide, 128-row swizzled box: 16 KB
+
+template <int D>
+struct Cfg {
+  static constexpr int kChunks = D / 64;
+  static constexpr int kTileBytes = kBM * D * 2;  // a Q, K, V or O tile
+  static constexpr int kStages = D == 128 ? 4 : 8;
+  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 1 + 1;
+  static constexpr int kSmemTiles = (kQTiles + kStages) * kTileBytes;
+  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 1024;
+  static constexpr uint32_t kColO = 256;
+};
+
+struct FwdParams {
+  float* lse;           // [BH][N] or nullptr
+  int N;                // sequence length
+  int n_qblk;           // ceil(N / 256)
+  int n_kv;             // ceil(N / 128)
+  float scale_log2;     // scale * log2(e)
+  uint64_t timeout_ns;  // bound on every wait
+  uint32_t debug;       // bit 0: stall the softmax warps on a barrier nobody signals
+};
+
+__device__ uint32_t g_device_status;
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                  const FwdParams p) {
+  using C = Cfg<D>;
+  constexpr int S = C::kStages;
+  constexpr int TB = C::kTileBytes;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;                  // kQTiles tiles (reused as O staging)
+  uint8_t* sKV = smem + kQTiles * TB;  // S stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemTiles);
+  uint64_t* q_full = bars;            // [2]   TMA -> MMA
+  uint64_t* kv_full = bars + 2;       // [S]   TMA -> MMA
+  uint64_t* kv_empty = kv_full + S;   // [S]   MMA -> TMA
+  uint64_t* s_full = kv_empty + S;    // [2]   MMA -> softmax
+  uint64_t* p_full = s_full + 2;      // [2]   softmax -> MMA (128 arrivals)
+  uint64_t* o_full = p_full + 2;      // [2]   MMA -> epilogue
+  uint64_t* mma_done = o_full + 2;    // [1]   MMA -> itself, before TMEM release
+  uint64_t* never = mma_done + 1;     // [1]   debug: nothing arrives here
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* status = &g_device_status;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x / p.n_qblk;
+  // heaviest query block of a head first (causal rows near the end see the most keys)
+  const int qblk = p.n_qblk - 1 - static_cast<int>(blockIdx.x % p.n_qblk);
+  const int q0 = qblk * kQTiles * kBM;
+  int kv_end = p.n_kv;
+  if (CAUSAL) kv_end = min(p.n_kv, (min(q0 + kQTiles * kBM, p.N) - 1) / kBN + 1);
+  const int n_iter = kv_end;  // KV tiles visited, from kv_end-1 down to 0
+  const uint64_t tmo = p.timeout_ns;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&q_full[0], 1);
+    mbar_init(&q_full[1], 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], kBM);
+      mbar_init(&o_full[t], 1);
+    }
+    mbar_init(mma_done, 1);
+    mbar_init(never, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmO);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      bool ok = true;
+      mbar_arrive_expect_tx(&q_full[0], TB);
+      for (int c = 0; c < C::kChunks; ++c)
+        tma_load_3d(sQ + c * kChunkBytes, &tmQ, &q_full[0], c * 64, q0, bh);
+      int i = 0;  // loads issued into the ring, in consumption order K0 V0 K1 V1 ...
+      for (int it = 0; it < n_iter && ok; ++it) {
+        const int j = kv_end - 1 - it;
+        for (int kv = 0; kv < 2; ++kv) {
+          const int s = i % S;
+          const uint32_t ph = static_cast<uint32_t>(i / S) & 1u;
+          ok = mbar_wait(&kv_empty[s], ph ^ 1u, abort_flag, status, tmo);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&kv_full[s], TB);
+          const CUtensorMap* m = kv == 0 ? &tmK : &tmV;
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d(sKV + s * TB + c * kChunkBytes, m, &kv_full[s], c * 64, j * kBN, bh);
+          ++i;
+          if (it == 0 && kv == 0) {
+            mbar_arrive_expect_tx(&q_full[1], TB);
+            for (int c = 0; c < C::kChunks; ++c)
+              tma_load_3d(sQ + TB + c * kChunkBytes, &tmQ, &q_full[1], c * 64, q0 + kBM, bh);
+          }
+        }
+      }
+      if (!ok) {
+        // Unwinding: wait for every copy already issued, so that none lands
+        // in shared memory after the CTA has ended.
+        for (int s = 0; s < S && s < i; ++s) {
+          const int last = s + ((i - 1 - s) / S) * S;
+          mbar_wait_drain(&kv_full[s], static_cast<uint32_t>(last / S) & 1u, tmo);
+        }
+        mbar_wait_drain(&q_full[0], 0, tmo);
+        if (i > 0) mbar_wait_drain(&q_full[1], 0, tmo);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(kBM, kBN, false);
+      constexpr uint32_t idO = idesc_bf16_f32(kBM, D, true);
+      const uint32_t sq = smem_addr(sQ);
+      const uint32_t skv = smem_addr(sKV);
+      // S_t = Q_t K^T: A = Q_t (K-major), B = K tile (K-major); 16 columns of
+      // d per instruction, 32 bytes apart inside each 128-byte swizzled row.
+      auto issue_s = [&](int t, int s) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
+          const uint64_t ad = sw128_desc(sq + t * TB + off, 16, 1024);
+          const uint64_t bd = sw128_desc(skv + s * TB + off, 16, 1024);
+          mma_ss(tmem + t * kBN, ad, bd, idS, kk > 0 ? 1u : 0u);
+        }
+      };
+      // O_t (+)= P_t V: A = P_t in TMEM (8 columns per 16 keys), B = V tile
+      // stored d-contiguous (MN-major): 16 keys = 2 KB apart, d halves 16 KB apart.
+      auto issue_pv = [&](int t, int s, bool accumulate) {
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint64_t bd = sw128_desc(skv + s * TB + kk * 2048, kChunkBytes, 1024);
+          mma_ts(tmem + C::kColO + t * D, tmem + t * kBN + kk * 8, bd, idO,
+                 (accumulate || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(&q_full[0], 0, abort_flag, status, tmo) &&
+                mbar_wait(&kv_full[0], 0, abort_flag, status, tmo);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        mma_commit(&s_full[0]);
+        ok = mbar_wait(&q_full[1], 0, abort_flag, status, tmo);
+      }
+      if (ok) {
+        tc_fence_after();
+        issue_s(1, 0);
+        mma_commit(&s_full[1]);
+        mma_commit(&kv_empty[0]);
+      }
+      for (int it = 0; it < n_iter && ok; ++it) {
+        const int iv = 2 * it + 1, ik = 2 * it + 2;
+        const int sv = iv % S, sk = ik % S;
+        const bool last = it == n_iter - 1;
+        if (!(ok = mbar_wait(&kv_full[sv], static_cast<uint32_t>(iv / S) & 1u, abort_flag, status, tmo))) break;
+        if (!(ok = mbar_wait(&p_full[0], static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo))) break;
+        tc_fence_after();
+        issue_pv(0, sv, it > 0);
+        if (last) {
+          mma_commit(&o_full[0]);
+        } else {
+          if (!(ok = mbar_wait(&kv_full[sk], static_cast<uint32_t>(ik / S) & 1u, abort_flag, status, tmo))) break;
+          tc_fence_after();
+          issue_s(0, sk);
+          mma_commit(&s_full[0]);
+        }
+        if (!(ok = mbar_wait(&p_full[1], static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo))) break;
+        tc_fence_after();
+        issue_pv(1, sv, it > 0);
+        mma_commit(&kv_empty[sv]);
+        if (last) {
+          mma_commit(&o_full[1]);
+        } else {
+          issue_s(1, sk);
+          mma_commit(&s_full[1]);
+          mma_commit(&kv_empty[sk]);
+        }
+      }
+      // every MMA issued here has finished before TMEM is released
+      mma_commit(mma_done);
+      mbar_wait_drain(mma_done, 0, tmo);
+    }
+  } else if (warp >= kSoftmaxWarp0) {
+    // ------------------------------------------------------------ softmax
+    const int t = (warp - kSoftmaxWarp0) >> 2;  // query tile of this warpgroup
+    const int wq = warp & 3;                    // TMEM lane quarter
+    const int r = wq * 32 + lane;               // row inside the tile
+    const int row = q0 + t * kBM + r;           // query index in the head
+    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_base + t * kBN;
+    const uint32_t tO = tmem + lane_base + C::kColO + t * D;
+    const float sl2 = p.scale_log2;
+    const int tile_first_row = q0 + t * kBM;
+    // last key this row may see
+    const int key_limit = CAUSAL ? min(row, p.N - 1) : p.N - 1;
+
+    float m_ref = -INFINITY;  // reference maximum, log2 units of scaled scores
+    float l_sum = 0.f;        // running denominator relative to m_ref
+    bool ok = true;
+    if (p.debug & 1u) {
+      ok = __all_sync(0xffffffffu, mbar_wait(never, 0, abort_flag, status, tmo));
+    }
+    for (int it = 0; it < n_iter && ok; ++it) {
+      const int j = kv_end - 1 - it;
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(&s_full[t], static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, sr[q]);
+      tmem_wait_ld();
+
+      const int kbase = j * kBN;
+      const bool masked = (kbase + kBN > p.N) || (CAUSAL && kbase + kBN - 1 > tile_first_row);
+      if (masked) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (kbase + q * 32 + c > key_limit) sr[q][c] = __float_as_uint(-INFINITY);
+      }
+      // row maximum of the raw scores (scale > 0 keeps the argmax)
+      float mx[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(sr[k >> 1][(k & 1) * 16]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int k = q * 2 + (c >> 4);
+          if ((c & 15) != 0) mx[k] = fmaxf(mx[k], __uint_as_float(sr[q][c]));
+        }
+      const float m_tile =
+          fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+      // raise the reference maximum only when this tile exceeds it by > 2^8
+      const bool raise = m_tile > m_ref + kRescaleThreshold;
+      float alpha = 1.f;
+      if (raise) {
+        alpha = ex2_approx(m_ref - m_tile);  // 0 while m_ref is -inf
+        m_ref = m_tile;
+      }
+      const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
+      // p = 2^(x - m) as bf16 pairs, written over the first 64 columns of
+      // S_t in two halves so that only 32 packed registers are live at once.
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int qq = 0; qq < 2; ++qq) {
+          const int q = 2 * h + qq;
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[q][c]), sl2, neg_m));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(sr[q][c + 1]), sl2, neg_m));
+            ps[q] += p0 + p1;
+            pk[qq * 16 + (c >> 1)] = pack_bf16x2(p0, p1);
+          }
+        }
+        tmem_st32(tS + h * 32, pk);
+      }
+      l_sum = l_sum * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+      if (it > 0 && __any_sync(0xffffffffu, raise)) {
+        // O_t holds the product through the previous tile (that MMA finished
+        // before S_t of this tile was committed): rescale it in place, after
+        // the scores have left the registers.
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+          tmem_st32(tO + c * 32, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[t]);
+    }
+
+    // ------------------------------------------------------------ epilogue
+    if (ok) ok = mbar_wait(&o_full[t], 0, abort_flag, status, tmo);
+    const bool failed = named_bar_or(1 + t, kBM, !ok);
+    if (!failed) {
+      tc_fence_after();
+      const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
+      if (p.lse != nullptr && row < p.N) {
+        const float lse2 = l_sum > 0.f ? m_ref + log2f(l_sum) : -INFINITY;
+        p.lse[static_cast<size_t>(bh) * p.N + row] = lse2 * 0.69314718055994530942f;
+      }
+      // O_t / l -> bf16 -> the Q_t buffer (no MMA reads it any more), laid
+      // out as the 128-byte-swizzled boxes the store tensor map expects.
+      uint8_t* stage = sQ + t * TB;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + c * 32, o);
+        tmem_wait_ld();
+        uint8_t* rowp = stage + (c >> 1) * kChunkBytes + r * 128;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(o[8 * g + 0]) * inv_l, __uint_as_float(o[8 * g + 1]) * inv_l);
+          v.y = pack_bf16x2(__uint_as_float(o[8 * g + 2]) * inv_l, __uint_as_float(o[8 * g + 3]) * inv_l);
+          v.z = pack_bf16x2(__uint_as_float(o[8 * g + 4]) * inv_l, __uint_as_float(o[8 * g + 5]) * inv_l);
+          v.w = pack_bf16x2(__uint_as_float(o[8 * g + 6]) * inv_l, __uint_as_float(o[8 * g + 7]) * inv_l);
+          const int gran = ((c & 1) * 4 + g) ^ (r & 7);
+          *reinterpret_cast<uint4*>(rowp + gran * 16) = v;
+        }
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1 + t, kBM);
+      if (r == 0 && tile_first_row < p.N) {
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_store_3d(&tmO, stage + c * kChunkBytes, c * 64, tile_first_row, bh);
+        bulk_commit_group();
+        bulk_wait_group_read0();
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+unsigned int g_debug_flags = 0;
+unsigned long long g_timeout_ns = 0;
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
+
+fa_status cuda_fail(cudaError_t e, const char* what) {
+  snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", what, cudaGetErrorString(e));
+  return FA_ERR_CUDA;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// [BH][N][d] bf16 viewed as a 3-D tensor (d fastest); boxes of 64 x 128 x 1
+// with the 128-byte swizzle.  Rows past N read as zero and are not stored.
+bool make_map(CUtensorMap* map, const void* base, int d, int N, int BH) {
+  auto enc = encode_tiled();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kBM), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+struct DeviceInfo {
+  bool checked = false;
+  bool sm100 = false;
+  bool attr_set[4] = {false, false, false, false};
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_dev_mutex;
+
+template <int D, bool CAUSAL>
+fa_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                 const CUtensorMap& mo, const FwdParams& prm, int BH, cudaStream_t stream,
+                 DeviceInfo& dev) {
+  constexpr int slot = (D == 128 ? 2 : 0) + (CAUSAL ? 1 : 0);
+  auto kern = fa_fwd_kernel<D, CAUSAL>;
+  if (!dev.attr_set[slot]) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    dev.attr_set[slot] = true;
+  }
+  const long long grid = static_cast<long long>(BH) * prm.n_qblk;
+  kern<<<static_cast<unsigned>(grid), kThreads, Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, mo, prm);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+  return FA_OK;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" {
+
+const char* fa_version(void) { return "0.1.0"; }
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_NULL: return "FA_ERR_NULL: a required pointer is NULL";
+    case FA_ERR_SHAPE: return "FA_ERR_SHAPE: bad B/H/N, size overflow or non-finite scale";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: d must be 64 or 128, scale > 0, sm_100 GPU";
+    case FA_ERR_ALIGN: return "FA_ERR_ALIGN: Q/K/V/O need 16-byte, LSE 4-byte alignment";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA call or kernel launch failed";
+    case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT: a kernel gave up on a bounded wait";
+    case FA_ERR_ALIAS: return "FA_ERR_ALIAS: O or LSE overlaps an input or each other";
+  }
+  return "unknown fa_status";
+}
+
+const char* fa_last_cuda_error(void) { return fa::g_last_cuda_error; }
+
+void fa_set_debug(unsigned int flags, unsigned long long timeout_ns) {
+  fa::g_debug_flags = flags;
+  fa::g_timeout_ns = timeout_ns;
+}
+
+fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H,
+                 int N, int d, float scale, int causal, void* stream) {
+  using namespace fa;
+  if (!Q || !K || !V || !O) return FA_ERR_NULL;
+  if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
+  if (!std::isfinite(scale)) return FA_ERR_SHAPE;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!(scale > 0.f)) return FA_ERR_UNSUPPORTED;
+  const long long BH = static_cast<long long>(B) * H;
+  const long long n_qblk = (static_cast<long long>(N) + kQTiles * kBM - 1) / (kQTiles * kBM);
+  if (BH > (1ll << 30) || BH * n_qblk > 0x7fffffffll) return FA_ERR_SHAPE;
+  auto mis16 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) != 0; };
+  if (mis16(Q) || mis16(K) || mis16(V) || mis16(O)) return FA_ERR_ALIGN;
+  if (LSE && (reinterpret_cast<uintptr_t>(LSE) & 3u) != 0) return FA_ERR_ALIGN;
+  const size_t nbytes = static_cast<size_t>(BH) * N * d * 2;
+  const size_t lbytes = static_cast<size_t>(BH) * N * 4;
+  if (overlaps(O, nbytes, Q, nbytes) || overlaps(O, nbytes, K, nbytes) ||
+      overlaps(O, nbytes, V, nbytes))
+    return FA_ERR_ALIAS;
+  if (LSE && (overlaps(LSE, lbytes, Q, nbytes) || overlaps(LSE, lbytes, K, nbytes) ||
+              overlaps(LSE, lbytes, V, nbytes) || overlaps(LSE, lbytes, O, nbytes)))
+    return FA_ERR_ALIAS;
+
+  int dev_id = 0;
+  cudaError_t e = cudaGetDevice(&dev_id);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev_id < 0 || dev_id >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  DeviceInfo* dev;
+  {
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    dev = &g_devices[dev_id];
+    if (!dev->checked) {
+      int major = 0;
+      e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev_id);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+      dev->sm100 = (major == 10);
+      dev->checked = true;
+    }
+  }
+  if (!dev->sm100) return FA_ERR_UNSUPPORTED;
+
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_map(&mq, Q, d, N, static_cast<int>(BH)) || !make_map(&mk, K, d, N, static_cast<int>(BH)) ||
+      !make_map(&mv, V, d, N, static_cast<int>(BH)) || !make_map(&mo, O, d, N, static_cast<int>(BH))) {
+    snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed");
+    return FA_ERR_CUDA;
+  }
+  FwdParams prm;
+  prm.lse = LSE;
+  prm.N = N;
+  prm.n_qblk = static_cast<int>(n_qblk);
+  prm.n_kv = (N + kBN - 1) / kBN;
+  prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
+  prm.timeout_ns = g_timeout_ns ? g_timeout_ns : kDefaultTimeoutNs;
+  prm.debug = g_debug_flags;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int bh = static_cast<int>(BH);
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  if (d == 128)
+    return causal ? launch<128, true>(mq, mk, mv, mo, prm, bh, st, *dev)
+                  : launch<128, false>(mq, mk, mv, mo, prm, bh, st, *dev);
+  return causal ? launch<64, true>(mq, mk, mv, mo, prm, bh, st, *dev)
+                : launch<64, false>(mq, mk, mv, mo, prm, bh, st, *dev);
+}
+
+fa_status fa_get_device_status(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return fa::cuda_fail(e, "cudaStreamSynchronize");
+  uint32_t v = 0;
+  e = cudaMemcpyFromSymbol(&v, fa::g_device_status, sizeof(v));
+  if (e != cudaSuccess) return fa::cuda_fail(e, "cudaMemcpyFromSymbol");
+  if (v != 0) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbol(fa::g_device_status, &zero, sizeof(zero));
+    if (e != cudaSuccess) return fa::cuda_fail(e, "cudaMemcpyToSymbol");
+    return FA_ERR_DEVICE_TIMEOUT;
+  }
+  return FA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,159 @@
+"""ctypes binding of libfa.so (include/fa.h): argument marshalling only.
+
+Every step of the attention forward runs in the library's CUDA kernel; this
+module checks tensor properties, passes raw pointers and the current CUDA
+stream, and turns status codes into exceptions.  There is no fallback: if the
+library is missing or the device is not an sm_100 GPU, calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libfa.so"
+
+FA_OK = 0
+FA_ERR_DEVICE_TIMEOUT = 6
+
+
+class FAError(RuntimeError):
+    """A libfa call returned a non-OK status."""
+
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+def library_path() -> str:
+    return os.environ.get("FA_LIBRARY", os.path.join(_HERE, _LIB_NAME))
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} not found: build the CUDA library first "
+            "(python -m exact_softmax_attention_02_b200.build)")
+    lib = ctypes.CDLL(path)
+    vp, c_int, c_float = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_float, c_int, vp]
+    lib.fa_fwd.restype = c_int
+    lib.fa_status_string.argtypes = [c_int]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_get_device_status.argtypes = [vp]
+    lib.fa_get_device_status.restype = c_int
+    lib.fa_last_cuda_error.argtypes = []
+    lib.fa_last_cuda_error.restype = ctypes.c_char_p
+    lib.fa_set_debug.argtypes = [ctypes.c_uint, ctypes.c_ulonglong]
+    lib.fa_set_debug.restype = None
+    lib.fa_version.argtypes = []
+    lib.fa_version.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _check(status: int):
+    if status != FA_OK:
+        lib = _load()
+        msg = lib.fa_status_string(status).decode()
+        detail = lib.fa_last_cuda_error().decode()
+        raise FAError(status, f"{msg}{' (' + detail + ')' if detail else ''}")
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+           lse: torch.Tensor | None = None, scale: float | None = None,
+           causal: bool = False, stream=None) -> None:
+    """Launch the fused forward: o = softmax(scale q k^T [causal]) v, lse.
+
+    q, k, v, o: CUDA bfloat16 [B, H, N, d], contiguous (d = 64 or 128).
+    lse: CUDA float32 [B, H, N] contiguous, or None.
+    scale: defaults to 1/sqrt(d).  Asynchronous on ``stream`` (default: the
+    current stream).
+    """
+    lib = _load()
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if t.dim() != 4:
+            raise ValueError(f"{name} must be [B, H, N, d]")
+    if not (q.shape == k.shape == v.shape == o.shape):
+        raise ValueError(f"shape mismatch: q{tuple(q.shape)} k{tuple(k.shape)} "
+                         f"v{tuple(v.shape)} o{tuple(o.shape)}")
+    B, H, N, d = q.shape
+    lse_ptr = None
+    if lse is not None:
+        if lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous():
+            raise ValueError("lse must be a contiguous CUDA float32 tensor")
+        if tuple(lse.shape) != (B, H, N):
+            raise ValueError(f"lse must be [B, H, N] = {(B, H, N)}")
+        lse_ptr = lse.data_ptr()
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    _check(lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_ptr,
+                      B, H, N, d, float(scale), int(bool(causal)), _stream_handle(stream)))
+
+
+def attention_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                      scale: float | None = None, causal: bool = False,
+                      return_lse: bool = True, device=None):
+    """Allocate the outputs and run the forward.
+
+    CUDA inputs: outputs stay on their device.  CPU inputs (ideally pinned):
+    they are copied to ``device`` (default cuda:current), the kernel runs
+    there, and O (and LSE) are copied back to pinned host memory; the call
+    returns after the copies have completed.
+    """
+    on_host = not q.is_cuda
+    if on_host:
+        dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        q = q.to(dev, non_blocking=True)
+        k = k.to(dev, non_blocking=True)
+        v = v.to(dev, non_blocking=True)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if return_lse else None
+    fa_fwd(q, k, v, o, lse, scale=scale, causal=causal)
+    if on_host:
+        o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        o_h.copy_(o, non_blocking=True)
+        lse_h = None
+        if lse is not None:
+            lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+            lse_h.copy_(lse, non_blocking=True)
+        torch.cuda.current_stream(o.device).synchronize()
+        return (o_h, lse_h) if return_lse else o_h
+    return (o, lse) if return_lse else o
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and read-and-clear the library's device status."""
+    return _load().fa_get_device_status(_stream_handle(stream))
+
+
+def set_debug(flags: int = 0, timeout_ns: int = 0) -> None:
+    """Test hook of include/fa.h (fa_set_debug)."""
+    _load().fa_set_debug(int(flags), int(timeout_ns))
+
+
+def version() -> str:
+    return _load().fa_version().decode()

@@ -1,0 +1,106 @@
+/*
+ * fa.h -- C ABI of libfa.so: exact softmax attention forward on B200 (sm_100a).
+ *
+ * The operation is the dense attention definition O = softmax(Q K^T / sqrt(d)) V
+ * (lihaoran.work, "FlashAttention: the intermediate matrix comes first", the
+ * opening formula), computed in one fused pass that keeps per-row running
+ * statistics -- the maximum m, the denominator l and the unnormalised
+ * numerator u -- and rescales them whenever a later key tile raises the
+ * maximum (liminalml.com "FlashAttention", the block update and "output u/l"
+ * after the final block; interactiveml.org "FlashAttention saves the matrix,
+ * not the quadratic work", the three sufficient statistics).  The N x N score
+ * matrix never reaches global memory (sadullah.online "Flash Attention
+ * Explained", fused tiled computation).
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors are dense, row-major, in device memory owned by the caller:
+ *       Q, K, V, O : bfloat16 [B][H][N][d]   (d fastest)
+ *       LSE        : float32  [B][H][N]
+ *   - Calls are asynchronous on the given stream (a cudaStream_t passed as
+ *     void*; NULL = the legacy default stream).  Nothing is valid until the
+ *     stream has been synchronised.
+ *   - The library never allocates device memory.
+ *   - Errors are returned as fa_status; argument errors are reported before
+ *     anything is launched.  Device-side failures (a bounded wait that gave
+ *     up) are reported by fa_get_device_status().
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fa_status {
+  FA_OK = 0,
+  FA_ERR_NULL = 1,            /* a required pointer is NULL                       */
+  FA_ERR_SHAPE = 2,           /* B, H or N < 1, sizes overflow, or scale not finite */
+  FA_ERR_UNSUPPORTED = 3,     /* d not in {64, 128}, scale <= 0, or not an sm_100 GPU */
+  FA_ERR_ALIGN = 4,           /* a pointer is not 16-byte aligned (LSE: 4-byte)   */
+  FA_ERR_CUDA = 5,            /* a CUDA runtime/driver call or the launch failed  */
+  FA_ERR_DEVICE_TIMEOUT = 6,  /* a kernel gave up on a bounded wait               */
+  FA_ERR_ALIAS = 7            /* O or LSE overlaps an input or each other         */
+} fa_status;
+
+/*
+ * fa_fwd -- O = softmax(scale * Q K^T [+ causal mask]) V, and its log-sum-exp.
+ *
+ *   Q, K, V  device, bf16 [B][H][N][d], read only; they may alias each other.
+ *   O        device, bf16 [B][H][N][d], written:
+ *              O[b,h,i,:] = sum_j w_ij V[b,h,j,:] / sum_j w_ij,
+ *              w_ij = exp(scale * <Q[b,h,i,:], K[b,h,j,:]> - m_i)
+ *            over the allowed keys j (all j, or j <= i when causal != 0),
+ *            rounded to bf16 (round to nearest even).
+ *   LSE      device, fp32 [B][H][N], written: ln sum_j exp(scale * <q_i, k_j>)
+ *            over the allowed keys (natural log of the scaled scores).  May be
+ *            NULL, in which case it is not written.
+ *   B, H, N  batch, heads, sequence length (queries and keys), each >= 1;
+ *            any N is accepted (ragged last tile is masked).
+ *   d        head width: 64 or 128.
+ *   scale    positive finite multiplier of the dot product (1/sqrt(d) for the
+ *            standard definition).
+ *   causal   0: every key is allowed; nonzero: query i sees keys j <= i.
+ *   stream   cudaStream_t (as void*) on which the kernel is launched.
+ *
+ * Q, K, V and O must be 16-byte aligned; LSE 4-byte aligned.  O and LSE must
+ * not overlap the inputs or each other.  Returns FA_OK once the kernel is
+ * enqueued.
+ */
+fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H,
+                 int N, int d, float scale, int causal, void* stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fa_status_string(fa_status status);
+
+/*
+ * fa_get_device_status -- synchronise `stream`, then read and clear the
+ * device status word of the current device.  Returns FA_ERR_DEVICE_TIMEOUT
+ * if any kernel launched by this library gave up on a bounded wait since the
+ * last call (its outputs are then undefined), FA_ERR_CUDA if the
+ * synchronisation failed, FA_OK otherwise.
+ */
+fa_status fa_get_device_status(void* stream);
+
+/* Message of the last CUDA error seen by this library in the calling thread
+ * ("" if none).  Static thread-local storage; valid until the next call. */
+const char* fa_last_cuda_error(void);
+
+/*
+ * fa_set_debug -- test hook.  Applies to kernels launched afterwards from any
+ * thread.  timeout_ns: how long a bounded wait inside a kernel may spin
+ * before it gives up (0 = default, 2 s).  flags bit 0: make the softmax
+ * warps of every CTA wait on a barrier that nothing arrives at, so that the
+ * wait runs out, the CTA unwinds without trapping, and
+ * fa_get_device_status() reports FA_ERR_DEVICE_TIMEOUT.  flags = 0 restores
+ * normal operation.
+ */
+void fa_set_debug(unsigned int flags, unsigned long long timeout_ns);
+
+/* Library version as "major.minor.patch" (static string). */
+const char* fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

@@ -1,0 +1,110 @@
+"""The C-ABI library without a GPU: it loads, exports every declared symbol,
+and rejects bad arguments before anything is launched.
+
+Only argument combinations that fail validation are passed (fake pointers
+never reach a launch), so these tests are safe on any machine.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+LIB = os.path.join(ROOT, "exact_softmax_attention_02_b200", "libfa.so")
+
+FA_OK, FA_ERR_NULL, FA_ERR_SHAPE, FA_ERR_UNSUPPORTED, FA_ERR_ALIGN = 0, 1, 2, 3, 4
+FA_ERR_CUDA, FA_ERR_DEVICE_TIMEOUT, FA_ERR_ALIAS = 5, 6, 7
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(LIB):
+        from exact_softmax_attention_02_b200.build import build
+
+        build()
+    lib = ctypes.CDLL(LIB)
+    vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, cf, ci, vp]
+    lib.fa_fwd.restype = ci
+    lib.fa_status_string.argtypes = [ci]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_version.restype = ctypes.c_char_p
+    return lib
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("fa_fwd", "fa_status_string", "fa_get_device_status"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"libfa.so does not export {name}"
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        s = lib.fa_status_string(code).decode()
+        assert s.startswith("FA_")
+    assert lib.fa_status_string(99).decode() == "unknown fa_status"
+    assert re.match(r"^\d+\.\d+\.\d+$", lib.fa_version().decode())
+
+
+A = 0x10000000  # fake, 16-byte-aligned "device" addresses: never dereferenced
+MB = 1 << 20
+
+
+def call(lib, q=A, k=A + 64 * MB, v=A + 128 * MB, o=A + 192 * MB, lse=A + 256 * MB,
+         B=1, H=1, N=128, d=64, scale=0.125, causal=0):
+    return lib.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, None)
+
+
+def test_null_pointers(lib):
+    assert call(lib, q=None) == FA_ERR_NULL
+    assert call(lib, k=None) == FA_ERR_NULL
+    assert call(lib, v=None) == FA_ERR_NULL
+    assert call(lib, o=None) == FA_ERR_NULL
+
+
+@pytest.mark.parametrize("B,H,N", [(0, 1, 128), (1, 0, 128), (1, 1, 0), (-1, 1, 128), (1, 1, -5),
+                                   (1 << 20, 1 << 20, 128)])
+def test_bad_shapes(lib, B, H, N):
+    assert call(lib, B=B, H=H, N=N) == FA_ERR_SHAPE
+
+
+@pytest.mark.parametrize("d", [0, 32, 96, 256, 65])
+def test_unsupported_head_width(lib, d):
+    assert call(lib, d=d) == FA_ERR_UNSUPPORTED
+
+
+def test_bad_scale(lib):
+    assert call(lib, scale=float("nan")) == FA_ERR_SHAPE
+    assert call(lib, scale=float("inf")) == FA_ERR_SHAPE
+    assert call(lib, scale=0.0) == FA_ERR_UNSUPPORTED
+    assert call(lib, scale=-0.5) == FA_ERR_UNSUPPORTED
+
+
+def test_misaligned(lib):
+    assert call(lib, q=A + 8) == FA_ERR_ALIGN
+    assert call(lib, v=A + 128 * MB + 2) == FA_ERR_ALIGN
+    assert call(lib, o=A + 192 * MB + 4) == FA_ERR_ALIGN
+    assert call(lib, lse=A + 256 * MB + 2) == FA_ERR_ALIGN
+
+
+def test_aliasing(lib):
+    # O overlapping an input
+    assert call(lib, o=A + 64) == FA_ERR_ALIAS
+    # LSE inside O
+    assert call(lib, lse=A + 192 * MB + 1024) == FA_ERR_ALIAS
+    # LSE overlapping V
+    assert call(lib, lse=A + 128 * MB) == FA_ERR_ALIAS

@@ -1,0 +1,270 @@
+"""GPU parity: the CUDA forward through the C ABI against the float64 oracle.
+
+Tolerances: max |O_gpu - O_oracle| <= 2e-2, mean <= 2e-3 (bf16 output,
+N(0,1)-scale inputs) and max |LSE_gpu - LSE_oracle| <= 1e-3.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from exact_softmax_attention_02_b200.inputs import WORKLOADS, make_qkv, sample_rows
+from oracle import attention_rows
+
+pytestmark = pytest.mark.gpu
+
+O_MAX, O_MEAN, LSE_MAX = 2e-2, 2e-3, 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_ready():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from exact_softmax_attention_02_b200 import fa
+
+    fa._load()
+    yield
+    fa.set_debug(0, 0)
+
+
+def gpu_forward(q, k, v, causal, scale=None, with_lse=True, stream=None):
+    from exact_softmax_attention_02_b200 import fa
+
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    o = torch.full_like(qd, float("nan"))  # canary: unwritten elements stay NaN
+    lse = torch.full(qd.shape[:3], float("nan"), device="cuda") if with_lse else None
+    fa.fa_fwd(qd, kd, vd, o, lse, scale=scale, causal=causal, stream=stream)
+    assert fa.device_status(stream) == 0
+    return o.cpu(), (lse.cpu() if with_lse else None)
+
+
+def compare(q, k, v, causal, rows, scale=None, o_max=O_MAX, o_mean=O_MEAN, lse_max=LSE_MAX):
+    d = q.shape[-1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o, lse = gpu_forward(q, k, v, causal, scale=scale)
+    rows_np = rows.numpy() if isinstance(rows, torch.Tensor) else np.asarray(rows)
+    ro, rl = attention_rows(q.float().numpy(), k.float().numpy(), v.float().numpy(),
+                            scale, causal, rows_np)
+    b, h, i = rows_np[:, 0], rows_np[:, 1], rows_np[:, 2]
+    go = o.double().numpy()[b, h, i]
+    gl = lse.double().numpy()[b, h, i]
+    assert np.all(np.isfinite(go)) and np.all(np.isfinite(gl))
+    err = np.abs(go - ro)
+    lerr = np.abs(gl - rl)
+    assert err.max() <= o_max, f"max |dO| = {err.max():.3e}"
+    assert err.mean() <= o_mean, f"mean |dO| = {err.mean():.3e}"
+    assert lerr.max() <= lse_max, f"max |dLSE| = {lerr.max():.3e}"
+    return o, lse, err, lerr
+
+
+def every_row(B, H, N):
+    return sample_rows(B, H, N, 0, 0)
+
+
+# ---------------------------------------------------------------------------
+# every row, several tiles, ragged tails
+# ---------------------------------------------------------------------------
+
+def test_plumbing_case_every_row():
+    w = WORKLOADS["b1h1n256d64"]
+    q, k, v = make_qkv(w.B, w.H, w.N, w.d, w.seed)
+    o, lse, _, _ = compare(q, k, v, w.causal, every_row(w.B, w.H, w.N))
+    assert not torch.isnan(o).any() and not torch.isnan(lse).any()
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 2, 127, 128, 129, 255, 256, 257, 300, 640, 1000])
+def test_every_row_shapes(d, causal, N):
+    B, H = (2, 3) if N <= 300 else (1, 2)
+    q, k, v = make_qkv(B, H, N, d, seed=N * 7 + d + int(causal))
+    o, lse, _, _ = compare(q, k, v, causal, every_row(B, H, N))
+    assert not torch.isnan(o).any() and not torch.isnan(lse).any()
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_peaked_rows_stress_rescaling(d):
+    """Q ~ N(0, 4^2): sharply peaked rows whose maximum moves between tiles."""
+    q, k, v = make_qkv(1, 4, 1024, d, seed=11, q_std=4.0)
+    compare(q, k, v, True, every_row(1, 4, 1024))
+    compare(q, k, v, False, every_row(1, 4, 1024))
+
+
+def test_large_score_magnitudes():
+    """Scores of several hundred: exponents must stay bounded (max subtraction)."""
+    q, k, v = make_qkv(1, 2, 512, 128, seed=5, q_std=20.0, k_std=3.0)
+    compare(q, k, v, True, every_row(1, 2, 512), lse_max=5e-3)
+
+
+def test_custom_scale_and_no_lse():
+    q, k, v = make_qkv(1, 2, 384, 64, seed=21)
+    compare(q, k, v, False, every_row(1, 2, 384), scale=0.37)
+    o_with, _ = gpu_forward(q, k, v, True, scale=0.2)
+    o_without, _ = gpu_forward(q, k, v, True, scale=0.2, with_lse=False)
+    assert torch.equal(o_with, o_without)
+
+
+def test_aliased_inputs_and_side_stream():
+    q, _, _ = make_qkv(1, 2, 512, 128, seed=8)
+    s = torch.cuda.Stream()
+    from exact_softmax_attention_02_b200 import fa
+
+    qd = q.cuda()
+    o = torch.empty_like(qd)
+    lse = torch.empty(qd.shape[:3], device="cuda")
+    with torch.cuda.stream(s):
+        fa.fa_fwd(qd, qd, qd, o, lse, causal=True, stream=s)
+    assert fa.device_status(s) == 0
+    rows = every_row(1, 2, 512).numpy()
+    ro, rl = attention_rows(q.float().numpy(), q.float().numpy(), q.float().numpy(),
+                            1 / math.sqrt(128), True, rows)
+    go = o.cpu().double().numpy()[rows[:, 0], rows[:, 1], rows[:, 2]]
+    assert np.abs(go - ro).max() <= O_MAX
+    assert np.abs(lse.cpu().double().numpy().ravel() - rl).max() <= LSE_MAX
+
+
+def test_deterministic():
+    q, k, v = make_qkv(2, 4, 777, 128, seed=3)
+    a, la = gpu_forward(q, k, v, True)
+    b, lb = gpu_forward(q, k, v, True)
+    assert torch.equal(a, b) and torch.equal(la, lb)
+
+
+def test_host_buffers_round_trip():
+    from exact_softmax_attention_02_b200 import fa
+
+    q, k, v = make_qkv(1, 2, 256, 64, seed=4)
+    q, k, v = (t.pin_memory() for t in (q, k, v))
+    o, lse = fa.attention_forward(q, k, v, causal=True)
+    assert not o.is_cuda and not lse.is_cuda
+    od, ld = gpu_forward(q, k, v, True)
+    assert torch.equal(o, od) and torch.equal(lse, ld)
+
+
+# ---------------------------------------------------------------------------
+# the pages' worked examples, embedded in one real 128-key tile
+# ---------------------------------------------------------------------------
+
+def _example_tile():
+    """d = 64, scale = 1.  Score(i, j) = alpha_i a_j + r_j + membership:
+
+    component 0 carries a_j (0 or 1000), component 1 carries r_j, component
+    3+g is 0 for keys of group g and -30000 for every other key, and query
+    rows of group g have a 1 there, so foreign keys get weight exactly 0.
+    Values are value_j * e0.
+    """
+    N, d = 128, 64
+    q = torch.zeros(1, 1, N, d)
+    k = torch.zeros(1, 1, N, d)
+    v = torch.zeros(1, 1, N, d)
+    groups = [
+        # (alpha, [(a_j, r_j, value_j)])   -- source of each group:
+        (0.0, [(0, 0, 10), (0, 1, 20), (0, 2, 30)]),        # lihaoran.work "Check three scores"
+        (1.0, [(1000, 0, 10), (1000, 1, 20), (1000, 2, 30)]),  # same, every score + 1000
+        (1.0, [(0, 1, 2), (0, 2, -1), (1000, 1, 4), (1000, 2, 8)]),  # liminalml.com scalar example
+    ]
+    j = 0
+    members = []
+    for g, (alpha, keys) in enumerate(groups):
+        q[0, 0, g, 0] = alpha
+        q[0, 0, g, 1] = 1.0
+        q[0, 0, g, 3 + g] = 1.0
+        idx = []
+        for a, r, val in keys:
+            k[0, 0, j, 0] = a
+            k[0, 0, j, 1] = r
+            v[0, 0, j, 0] = val
+            idx.append(j)
+            j += 1
+        members.append(idx)
+    for g in range(len(groups)):
+        for jj in range(N):
+            if jj not in members[g]:
+                k[0, 0, jj, 3 + g] = -30000.0
+    return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+
+
+def test_worked_examples_inside_a_tile():
+    q, k, v = _example_tile()
+    o, lse = gpu_forward(q, k, v, False, scale=1.0)
+    e = math.e
+    three = (10 + 20 * e + 30 * e * e) / (1 + e + e * e)
+    four = (4 + 8 * e) / (1 + e)
+    expect = [
+        (three, math.log(1 + e + e * e)),
+        (three, 1000 + math.log(1 + e + e * e)),
+        (four, 1002 + math.log(1 + math.exp(-1))),
+    ]
+    for row, (val, lval) in enumerate(expect):
+        got = o[0, 0, row].double()
+        assert abs(got[0].item() - val) <= O_MAX
+        # within one bf16 step of the exact value
+        ulp = 2.0 ** (math.floor(math.log2(abs(val))) - 7)
+        assert abs(got[0].item() - val) <= ulp
+        assert torch.all(got[1:] == 0)
+        assert abs(lse[0, 0, row].item() - lval) <= LSE_MAX
+    assert round(o[0, 0, 0, 0].item(), 2) == round(25.752104, 2)
+
+
+def test_rescale_when_a_later_tile_raises_the_maximum():
+    """Three key tiles whose best scores are 5, 10, 30/29 (liminalml.com: a
+    larger maximum rescales numerator and denominator together)."""
+    N, d = 384, 64
+    q = torch.zeros(1, 1, N, d)
+    k = torch.zeros(1, 1, N, d)
+    v = torch.zeros(1, 1, N, d)
+    q[0, 0, :, 1] = 1.0
+    q[0, 0, :, 2] = 1.0
+    k[0, 0, :, 2] = -30000.0
+    picks = {256: (5.0, 1.0), 128: (10.0, 2.0), 0: (30.0, 3.0), 1: (29.0, 4.0)}
+    for j, (s, val) in picks.items():
+        k[0, 0, j, 1] = s
+        k[0, 0, j, 2] = 0.0
+        v[0, 0, j, 0] = val
+    q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
+    o, lse = gpu_forward(q, k, v, False, scale=1.0)
+    w = {j: math.exp(s - 30.0) for j, (s, _) in picks.items()}
+    z = sum(w.values())
+    expect = sum(w[j] * picks[j][1] for j in picks) / z
+    assert abs(o[0, 0, 0, 0].item() - expect) <= 1e-2
+    assert abs(lse[0, 0, 0].item() - (30.0 + math.log(z))) <= LSE_MAX
+
+
+# ---------------------------------------------------------------------------
+# the benchmark problems at full size, on sampled rows
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["b4h16n4096d64", "b2h16n8192d128_causal",
+                                  "b1h32n32768d128_causal_q4", "b1h8n131072d128_causal"])
+def test_full_size_sampled_rows(name):
+    w = WORKLOADS[name]
+    q, k, v = make_qkv(w.B, w.H, w.N, w.d, w.seed, w.q_std)
+    rows = sample_rows(w.B, w.H, w.N, w.sample_rows, w.seed)
+    o, lse, err, lerr = compare(q, k, v, w.causal, rows)
+    # properties that hold for every row, checked over the whole output
+    assert not torch.isnan(o).any() and not torch.isnan(lse).any()
+    assert torch.isfinite(o.float()).all()
+    assert (o.float().abs() <= v.float().abs().amax() + 1e-2).all()
+
+
+# ---------------------------------------------------------------------------
+# failure detection: a wait that runs out unwinds the kernel cleanly
+# ---------------------------------------------------------------------------
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    from exact_softmax_attention_02_b200 import fa
+
+    q, k, v = make_qkv(1, 2, 512, 128, seed=2)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    o = torch.empty_like(qd)
+    fa.set_debug(1, 20_000_000)  # stall the softmax warps; give up after 20 ms
+    try:
+        fa.fa_fwd(qd, kd, vd, o, None, causal=True)
+        assert fa.device_status() == fa.FA_ERR_DEVICE_TIMEOUT
+    finally:
+        fa.set_debug(0, 0)
+    assert fa.device_status() == 0  # status was cleared
+    # the context is still usable and results are right again
+    compare(q, k, v, True, every_row(1, 2, 512))
