@@ -1,0 +1,448 @@
+"""Benchmark of the fused exact-attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one fa_fwd launch over the whole problem (every query row of
+every head).  The default problem is B=2, H=16, N=8192, d=128, causal, bf16
+inputs from N(0,1) with seed 2; inputs plus output (268 MB) exceed the 126 MB
+L2, so no flush is inserted between steps.  FLOPs are counted as
+4*B*H*N^2*d, halved for causal.
+
+Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
+and a device synchronise on both sides, measured with CUDA events on the
+launching stream; the time is the maximum over ranks.  With N > 1 (launched
+by torch.distributed.run) every rank runs the same problem on its own seeded
+inputs: weak scaling with no collective on the data path.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the float64 CPU
+oracle instead (the reference arm), on bounded row samples of the same
+problem; under torchrun only rank 0 runs it.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd TFLOP/s (bf16, 1×B200) and % of dense-BF16 tensor peak"
+DEFAULT_WORKLOAD = "b2h16n8192d128_causal"
+FALLBACK_PEAK_TFLOPS = 1590.0
+L2_BYTES = 126 * 1024 * 1024
+KERNEL_SOURCES = ["exact_softmax_attention_02_b200/csrc/fa_fwd.cu",
+                  "exact_softmax_attention_02_b200/csrc/sm100.cuh"]
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (host logic, covered by CPU gloo tests)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    """(rank, local_rank, world_size) from the torchrun environment."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def init_dist(world: int, backend: str):
+    import datetime
+
+    import torch.distributed as dist
+
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own inputs; rank 0 keeps the workload's seed."""
+    return seed + 7919 * rank
+
+
+def max_over_ranks(value: float, dist, device=None) -> float:
+    import torch
+
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, dist, device=None) -> float:
+    import torch
+
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def weak_scaling_value(flops_per_rank_step: float, world: int, steps: int, seconds: float) -> float:
+    """Whole-job TFLOP/s: all ranks' FLOPs over the slowest rank's time."""
+    return flops_per_rank_step * world * steps / seconds / 1e12
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only; no setting is changed)
+# ---------------------------------------------------------------------------
+
+_REASON_BITS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+    0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+    0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+    0x100: "display_clock_setting",
+}
+
+
+class ClockSampler:
+    """Polls SM clock, power and clock-event reasons from a thread."""
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._nvml = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML unavailable: report no clocks rather than guess
+            self._nvml = None
+
+    def _run(self):
+        n = self._nvml
+        while not self._stop.is_set():
+            try:
+                mhz = n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM)
+                try:
+                    reasons = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except Exception:
+                    reasons = n.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                util = n.nvmlDeviceGetUtilizationRates(self._h).gpu
+                self.samples.append((mhz, int(reasons), util))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        loaded = [s for s in self.samples if not (s[1] & 0x1)] or self.samples
+        mask = 0
+        for _, r, _ in loaded:
+            mask |= r
+        reasons = [name for bit, name in sorted(_REASON_BITS.items()) if mask & bit and bit != 0x1]
+        return {"sm_mhz": statistics.median(s[0] for s in loaded), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(loaded)}
+
+
+# ---------------------------------------------------------------------------
+# peaks and committed ncu evidence
+# ---------------------------------------------------------------------------
+
+def tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            peaks = json.load(f)
+        return float(peaks["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
+    except Exception:
+        return FALLBACK_PEAK_TFLOPS, "fallback (1.59 PFLOP/s, earlier measurement on this pool)"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary for this workload,
+    or None when there is none or the kernel source changed since."""
+    path = os.path.join(ROOT, "profiles", f"fa_fwd_{workload}_ncu.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            line = line.strip().lstrip("-* ")
+            for key in ("dram_bytes_per_launch", "kernel_source_sha256"):
+                if line.startswith(key + ":"):
+                    vals[key] = line.split(":", 1)[1].strip().strip("`")
+    if vals.get("kernel_source_sha256") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------------------
+# the oracle on host cores (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def blas_threads() -> int:
+    try:
+        import threadpoolctl
+
+        info = threadpoolctl.threadpool_info()
+        n = [i["num_threads"] for i in info if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample_time(w, q32, k32, v32, rows):
+    """Run the oracle on ``rows``; return (seconds, counted FLOPs)."""
+    from oracle import attention_rows, flops_for_rows
+
+    t0 = time.perf_counter()
+    attention_rows(q32, k32, v32, w.scale, w.causal, rows)
+    dt = time.perf_counter() - t0
+    return dt, flops_for_rows(rows, w.N, w.d, w.causal)
+
+
+def oracle_inputs(w, seed):
+    from exact_softmax_attention_02_b200.inputs import make_qkv
+
+    q, k, v = make_qkv(w.B, w.H, w.N, w.d, seed, w.q_std)
+    return q.float().numpy(), k.float().numpy(), v.float().numpy()
+
+
+def random_rows(w, count, seed):
+    import numpy as np
+
+    rng = np.random.default_rng(seed)
+    flat = rng.choice(w.B * w.H * w.N, size=min(count, w.B * w.H * w.N), replace=False)
+    return np.stack([flat // (w.H * w.N), (flat // w.N) % w.H, flat % w.N], axis=1)
+
+
+def cpu_baseline(w, seed, target_s: float = 12.0):
+    """Oracle throughput on a bounded random row sample, in TFLOP/s."""
+    q32, k32, v32 = oracle_inputs(w, seed)
+    n = 64
+    dt, _ = oracle_sample_time(w, q32, k32, v32, random_rows(w, n, seed + 1))
+    n = int(max(64, min(w.B * w.H * w.N, n * target_s / max(dt, 1e-3))))
+    rows = random_rows(w, n, seed + 2)
+    dt, flops = oracle_sample_time(w, q32, k32, v32, rows)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{len(rows)} random query rows of {w.name} (float64 numpy, "
+                      f"{dt:.1f} s; FLOPs counted 4*d per allowed key)"}
+
+
+# ---------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------
+
+def run_reference(args, w):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    q32, k32, v32 = oracle_inputs(w, w.seed)
+    budget_per_step = min(8.0, 150.0 / max(1, args.steps + args.warmup))
+    n = 32
+    dt, _ = oracle_sample_time(w, q32, k32, v32, random_rows(w, n, 1))
+    n = int(max(8, min(w.B * w.H * w.N, n * budget_per_step / max(dt, 1e-3))))
+    for i in range(args.warmup):
+        oracle_sample_time(w, q32, k32, v32, random_rows(w, n, 100 + i))
+    tot_t, tot_f = 0.0, 0.0
+    for i in range(args.steps):
+        dt, fl = oracle_sample_time(w, q32, k32, v32, random_rows(w, n, 1000 + i))
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    sample = (f"{n} random query rows of {w.name} per step (float64 numpy oracle; "
+              f"FLOPs counted 4*d per allowed key)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {**w.as_config(), "l2": "host oracle (no GPU)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, w):
+    import torch
+
+    from exact_softmax_attention_02_b200 import fa
+    from exact_softmax_attention_02_b200.inputs import make_qkv
+
+    rank, local_rank, world = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (B200); the CPU oracle arm is --impl reference")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = init_dist(world, "nccl")
+
+    seed = rank_seed(w.seed, rank)
+    q_h, k_h, v_h = make_qkv(w.B, w.H, w.N, w.d, seed, w.q_std)
+    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fa.fa_fwd(q, k, v, o, lse, scale=w.scale, causal=w.causal, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    if fa.device_status(stream) != 0:
+        raise RuntimeError("kernel reported a device timeout during warm-up")
+
+    sampler = ClockSampler(local_rank)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler.start()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    sampler.stop()
+    if fa.device_status(stream) != 0:
+        raise RuntimeError("kernel reported a device timeout in the timed region")
+    elapsed = t_start.elapsed_time(t_end) / 1e3
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    elapsed_max = max_over_ranks(elapsed, dist, dev)
+    avg_launch_s = max_over_ranks(sum(launch_ms) / len(launch_ms) / 1e3, dist, dev)
+
+    # end to end through the public API: pinned host inputs -> device -> O, LSE back to host
+    o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    q_p, k_p, v_p = (t.pin_memory() for t in (q_h, k_h, v_h))
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        fa.attention_forward(q_p, k_p, v_p, scale=w.scale, causal=w.causal, out=(o_h, lse_h))
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        fa.attention_forward(q_p, k_p, v_p, scale=w.scale, causal=w.causal, out=(o_h, lse_h))
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist, dev)
+    h2d = 3 * q.numel() * q.element_size()
+    d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+
+    clocks = sampler.summary()
+    value = weak_scaling_value(w.flops, world, args.steps, elapsed_max)
+    peak, peak_src = tensor_peak()
+    achieved = w.flops / avg_launch_s / 1e12
+    traffic = committed_traffic(w.name)
+    launches = int(sum_over_ranks(args.steps, dist, dev))
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, w.seed)
+
+    if dist is not None:
+        dist.barrier()
+    if rank == 0:
+        in_bytes = 4 * q.numel() * q.element_size() + lse.numel() * 4
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * elapsed_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 Q/K/V per rank)",
+            "config": {**w.as_config(), "parallelism": f"replicas{world}",
+                       "l2": (f"inputs+outputs {in_bytes / 1e6:.0f} MB > L2 126 MB, no flush"
+                              if in_bytes > L2_BYTES else "L2 not flushed (inputs < L2)")},
+            "pct_of_peak": 100.0 * value / world / peak,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": peak_src, "kernel": f"fa_fwd_kernel<{w.d},{str(w.causal).lower()}>",
+                         "kernel_source_sha256": kernel_source_hash()},
+            "e2e": {"value": weak_scaling_value(w.flops, world, e2e_steps, e2e_s), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    from exact_softmax_attention_02_b200.inputs import WORKLOADS
+
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.steps < 1:
+        ap.error("--steps must be >= 1")
+    w = WORKLOADS[args.workload]
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # not under torchrun: start one process per GPU the same way the
+        # harness does, on the loopback address
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+               f"--nproc-per-node={args.gpus}", "--master-addr=127.0.0.1",
+               "--master-port=29517", os.path.abspath(__file__), *(argv or sys.argv[1:])]
+        return subprocess.call(cmd)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

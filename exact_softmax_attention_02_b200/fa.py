@@ -116,33 +116,42 @@ def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
 
 def attention_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                       scale: float | None = None, causal: bool = False,
-                      return_lse: bool = True, device=None):
+                      return_lse: bool = True, device=None, out=None):
     """Allocate the outputs and run the forward.
 
     CUDA inputs: outputs stay on their device.  CPU inputs (ideally pinned):
-    they are copied to ``device`` (default cuda:current), the kernel runs
-    there, and O (and LSE) are copied back to pinned host memory; the call
+    they are copied to ``device`` (default: the current CUDA device), the
+    kernel runs there, and O (and LSE) are copied back to host memory -- into
+    ``out = (o_host, lse_host)`` when given (pinned buffers of the right shape
+    and dtype, reused across calls), else into new pinned tensors.  The call
     returns after the copies have completed.
     """
     on_host = not q.is_cuda
     if on_host:
-        dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        dev = torch.device(device) if device is not None else torch.device(
+            "cuda", torch.cuda.current_device())
         q = q.to(dev, non_blocking=True)
         k = k.to(dev, non_blocking=True)
         v = v.to(dev, non_blocking=True)
     o = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if return_lse else None
     fa_fwd(q, k, v, o, lse, scale=scale, causal=causal)
-    if on_host:
+    if not on_host:
+        return (o, lse) if return_lse else o
+    if out is not None:
+        o_h, lse_h = out
+        if tuple(o_h.shape) != tuple(o.shape) or o_h.dtype != o.dtype:
+            raise ValueError("out[0] must match O in shape and dtype")
+        if return_lse and (lse_h is None or tuple(lse_h.shape) != tuple(lse.shape)):
+            raise ValueError("out[1] must be a float32 [B, H, N] tensor")
+    else:
         o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-        o_h.copy_(o, non_blocking=True)
-        lse_h = None
-        if lse is not None:
-            lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
-            lse_h.copy_(lse, non_blocking=True)
-        torch.cuda.current_stream(o.device).synchronize()
-        return (o_h, lse_h) if return_lse else o_h
-    return (o, lse) if return_lse else o
+        lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True) if return_lse else None
+    o_h.copy_(o, non_blocking=True)
+    if return_lse:
+        lse_h.copy_(lse, non_blocking=True)
+    torch.cuda.current_stream(o.device).synchronize()
+    return (o_h, lse_h) if return_lse else o_h
 
 
 def device_status(stream=None) -> int:
