@@ -252,11 +252,15 @@ def random_rows(w, count, seed):
 def cpu_baseline(w, seed, target_s: float = 12.0):
     """Oracle throughput on a bounded random row sample, in TFLOP/s."""
     q32, k32, v32 = oracle_inputs(w, seed)
+    total = w.B * w.H * w.N
     n = 64
-    dt, _ = oracle_sample_time(w, q32, k32, v32, random_rows(w, n, seed + 1))
-    n = int(max(64, min(w.B * w.H * w.N, n * target_s / max(dt, 1e-3))))
-    rows = random_rows(w, n, seed + 2)
-    dt, flops = oracle_sample_time(w, q32, k32, v32, rows)
+    # grow the sample until one timed pass takes at least half the target
+    for attempt in range(8):
+        rows = random_rows(w, n, seed + 2 + attempt)
+        dt, flops = oracle_sample_time(w, q32, k32, v32, rows)
+        if dt >= 0.5 * target_s or n >= total:
+            break
+        n = int(min(total, n * min(16.0, max(2.0, target_s / max(dt, 1e-3)))))
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
             "kind": "oracle",
             "sample": f"{len(rows)} random query rows of {w.name} (float64 numpy, "

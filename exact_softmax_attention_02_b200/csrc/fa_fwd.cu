@@ -62,7 +62,18 @@ constexpr int kQTiles = 2;     // query tiles per CTA
 constexpr int kThreads = 384;  // 12 warps
 constexpr int kSoftmaxWarp0 = 4;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+#ifndef FA_EMU_PER32
+#define FA_EMU_PER32 0
+#endif
+// columns (of every 32) whose exponential runs on the FMA pipe instead of MUFU
+constexpr int kEmuPer32 = FA_EMU_PER32;
+static_assert(kEmuPer32 >= 0 && kEmuPer32 <= 32 && kEmuPer32 % 2 == 0, "even count per 32");
 constexpr uint32_t kTmemCols = 512;
+// wait sites reported in the device status word (bit 8 + site)
+enum : uint32_t {
+  kSiteKvEmpty = 0, kSiteQ = 1, kSiteKvFull = 2, kSiteS = 3, kSiteP = 4,  // 4..7: p_half[0..3]
+  kSiteO = 8, kSiteDebug = 9,
+};
 constexpr int kChunkBytes = kBM * 64 * 2;  // one 64-wide, 128-row swizzled box: 16 KB
 
 template <int D>
@@ -70,7 +81,7 @@ struct Cfg {
   static constexpr int kChunks = D / 64;
   static constexpr int kTileBytes = kBM * D * 2;  // a Q, K, V or O tile
   static constexpr int kStages = D == 128 ? 4 : 8;
-  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 1 + 1;
+  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 4 + 2 + 1 + 1;
   static constexpr int kSmemTiles = (kQTiles + kStages) * kTileBytes;
   static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 1024;
   static constexpr uint32_t kColO = 256;
@@ -79,6 +90,8 @@ struct Cfg {
 struct FwdParams {
   float* lse;           // [BH][N] or nullptr
   int N;                // sequence length
+  int BH;               // batch * heads
+  int group_heads;      // heads whose CTAs are scheduled together
   int n_qblk;           // ceil(N / 256)
   int n_kv;             // ceil(N / 128)
   float scale_log2;     // scale * log2(e)
@@ -87,6 +100,24 @@ struct FwdParams {
 };
 
 __device__ uint32_t g_device_status;
+
+// Optional phase trace (build with -DFA_TRACE): SM clock stamps of the MMA
+// issuer and of one thread per softmax warpgroup, for the first CTAs.
+#ifdef FA_TRACE
+constexpr int kTraceCtas = 16;
+constexpr int kTraceIters = 64;
+__device__ unsigned long long* g_trace;  // [kTraceCtas][4 roles][kTraceIters][8 events]
+#define FA_TRACE_MARK(role, iter, ev)                                                         \
+  do {                                                                                        \
+    if (g_trace != nullptr && blockIdx.x < kTraceCtas && (iter) < kTraceIters)                \
+      g_trace[((static_cast<size_t>(blockIdx.x) * 4 + (role)) * kTraceIters + (iter)) * 8 + \
+              (ev)] = clock64();                                                              \
+  } while (0)
+#else
+#define FA_TRACE_MARK(role, iter, ev) \
+  do {                                \
+  } while (0)
+#endif
 
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -107,8 +138,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* kv_full = bars + 2;       // [S]   TMA -> MMA
   uint64_t* kv_empty = kv_full + S;   // [S]   MMA -> TMA
   uint64_t* s_full = kv_empty + S;    // [2]   MMA -> softmax
-  uint64_t* p_full = s_full + 2;      // [2]   softmax -> MMA (128 arrivals)
-  uint64_t* o_full = p_full + 2;      // [2]   MMA -> epilogue
+  uint64_t* p_half = s_full + 2;      // [4]   softmax -> MMA, [2t+h] = half h of P_t (128 arrivals)
+  uint64_t* o_full = p_half + 4;      // [2]   MMA -> epilogue
   uint64_t* mma_done = o_full + 2;    // [1]   MMA -> itself, before TMEM release
   uint64_t* never = mma_done + 1;     // [1]   debug: nothing arrives here
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
@@ -117,9 +148,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x / p.n_qblk;
-  // heaviest query block of a head first (causal rows near the end see the most keys)
-  const int qblk = p.n_qblk - 1 - static_cast<int>(blockIdx.x % p.n_qblk);
+  // CTA order: heads in groups of p.group_heads; inside a group, query
+  // blocks from the heaviest (last rows: most keys when causal) to the
+  // lightest, cycling over the group's heads.  CTAs that run together then
+  // share the K/V of a few heads in L2, and light blocks end the grid.
+  const int per_group = p.group_heads * p.n_qblk;
+  const int grp = static_cast<int>(blockIdx.x) / per_group;
+  const int rem = static_cast<int>(blockIdx.x) % per_group;
+  const int grp_heads = min(p.group_heads, p.BH - grp * p.group_heads);
+  const int bh = grp * p.group_heads + rem % grp_heads;
+  const int qblk = p.n_qblk - 1 - rem / grp_heads;
   const int q0 = qblk * kQTiles * kBM;
   int kv_end = p.n_kv;
   if (CAUSAL) kv_end = min(p.n_kv, (min(q0 + kQTiles * kBM, p.N) - 1) / kBN + 1);
@@ -135,7 +173,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], kBM);
+      mbar_init(&p_half[2 * t], kBM);
+      mbar_init(&p_half[2 * t + 1], kBM);
       mbar_init(&o_full[t], 1);
     }
     mbar_init(mma_done, 1);
@@ -169,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kv = 0; kv < 2; ++kv) {
           const int s = i % S;
           const uint32_t ph = static_cast<uint32_t>(i / S) & 1u;
-          ok = mbar_wait(&kv_empty[s], ph ^ 1u, abort_flag, status, tmo);
+          ok = mbar_wait(&kv_empty[s], ph ^ 1u, abort_flag, status, tmo, kSiteKvEmpty);
           if (!ok) break;
           mbar_arrive_expect_tx(&kv_full[s], TB);
           const CUtensorMap* m = kv == 0 ? &tmK : &tmV;
@@ -214,21 +253,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // O_t (+)= P_t V: A = P_t in TMEM (8 columns per 16 keys), B = V tile
       // stored d-contiguous (MN-major): 16 keys = 2 KB apart, d halves 16 KB apart.
-      auto issue_pv = [&](int t, int s, bool accumulate) {
+      auto issue_pv = [&](int t, int s, bool accumulate, int half) {
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
+        for (int kk = half * (kBN / 32); kk < (half + 1) * (kBN / 32); ++kk) {
           const uint64_t bd = sw128_desc(skv + s * TB + kk * 2048, kChunkBytes, 1024);
           mma_ts(tmem + C::kColO + t * D, tmem + t * kBN + kk * 8, bd, idO,
                  (accumulate || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(&q_full[0], 0, abort_flag, status, tmo) &&
-                mbar_wait(&kv_full[0], 0, abort_flag, status, tmo);
+      bool ok = mbar_wait(&q_full[0], 0, abort_flag, status, tmo, kSiteQ) &&
+                mbar_wait(&kv_full[0], 0, abort_flag, status, tmo, kSiteKvFull);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
         mma_commit(&s_full[0]);
-        ok = mbar_wait(&q_full[1], 0, abort_flag, status, tmo);
+        ok = mbar_wait(&q_full[1], 0, abort_flag, status, tmo, kSiteQ);
       }
       if (ok) {
         tc_fence_after();
@@ -240,21 +279,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int iv = 2 * it + 1, ik = 2 * it + 2;
         const int sv = iv % S, sk = ik % S;
         const bool last = it == n_iter - 1;
-        if (!(ok = mbar_wait(&kv_full[sv], static_cast<uint32_t>(iv / S) & 1u, abort_flag, status, tmo))) break;
-        if (!(ok = mbar_wait(&p_full[0], static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo))) break;
+        const uint32_t ph_it = static_cast<uint32_t>(it) & 1u;
+        if (!(ok = mbar_wait(&kv_full[sv], static_cast<uint32_t>(iv / S) & 1u, abort_flag, status, tmo, kSiteKvFull))) break;
+        // P_t arrives in two halves of 64 keys (p_half[2t], p_half[2t+1]): the
+        // first four K-steps of the PV product start while the softmax is
+        // still on the second half.
+        if (!(ok = mbar_wait(&p_half[0], ph_it, abort_flag, status, tmo, kSiteP))) break;
+        FA_TRACE_MARK(0, it, 0);
         tc_fence_after();
-        issue_pv(0, sv, it > 0);
+        issue_pv(0, sv, it > 0, 0);
+        if (!(ok = mbar_wait(&p_half[1], ph_it, abort_flag, status, tmo, kSiteP + 1))) break;
+        tc_fence_after();
+        issue_pv(0, sv, true, 1);
+        FA_TRACE_MARK(0, it, 1);
         if (last) {
           mma_commit(&o_full[0]);
         } else {
-          if (!(ok = mbar_wait(&kv_full[sk], static_cast<uint32_t>(ik / S) & 1u, abort_flag, status, tmo))) break;
+          if (!(ok = mbar_wait(&kv_full[sk], static_cast<uint32_t>(ik / S) & 1u, abort_flag, status, tmo, kSiteKvFull))) break;
           tc_fence_after();
           issue_s(0, sk);
           mma_commit(&s_full[0]);
+          FA_TRACE_MARK(0, it, 2);
         }
-        if (!(ok = mbar_wait(&p_full[1], static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo))) break;
+        if (!(ok = mbar_wait(&p_half[2], ph_it, abort_flag, status, tmo, kSiteP + 2))) break;
+        FA_TRACE_MARK(0, it, 3);
         tc_fence_after();
-        issue_pv(1, sv, it > 0);
+        issue_pv(1, sv, it > 0, 0);
+        if (!(ok = mbar_wait(&p_half[3], ph_it, abort_flag, status, tmo, kSiteP + 3))) break;
+        tc_fence_after();
+        issue_pv(1, sv, true, 1);
+        FA_TRACE_MARK(0, it, 4);
         mma_commit(&kv_empty[sv]);
         if (last) {
           mma_commit(&o_full[1]);
@@ -262,6 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           issue_s(1, sk);
           mma_commit(&s_full[1]);
           mma_commit(&kv_empty[sk]);
+          FA_TRACE_MARK(0, it, 5);
         }
       }
       // every MMA issued here has finished before TMEM is released
@@ -286,18 +341,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     float l_sum = 0.f;        // running denominator relative to m_ref
     bool ok = true;
     if (p.debug & 1u) {
-      ok = __all_sync(0xffffffffu, mbar_wait(never, 0, abort_flag, status, tmo));
+      ok = __all_sync(0xffffffffu, mbar_wait(never, 0, abort_flag, status, tmo, kSiteDebug));
     }
     for (int it = 0; it < n_iter && ok; ++it) {
       const int j = kv_end - 1 - it;
       ok = __all_sync(0xffffffffu,
-                      mbar_wait(&s_full[t], static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo));
+                      mbar_wait(&s_full[t], static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteS));
       if (!ok) break;
+      const bool tr = lane == 0 && (warp & 3) == 0;
+      if (tr) FA_TRACE_MARK(1 + t, it, 0);
       tc_fence_after();
       uint32_t sr[4][32];
 #pragma unroll
       for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, sr[q]);
       tmem_wait_ld();
+      if (tr) FA_TRACE_MARK(1 + t, it, 1);
 
       const int kbase = j * kBN;
       const bool masked = (kbase + kBN > p.N) || (CAUSAL && kbase + kBN - 1 > tile_first_row);
@@ -308,20 +366,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 32; ++c)
             if (kbase + q * 32 + c > key_limit) sr[q][c] = __float_as_uint(-INFINITY);
       }
-      // row maximum of the raw scores (scale > 0 keeps the argmax)
+      // row maximum of the raw scores (scale > 0 keeps the argmax): eight
+      // independent chains of three-input maxima
       float mx[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(sr[k >> 1][(k & 1) * 16]);
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t* v = &sr[k >> 1][(k & 1) * 16];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int k = q * 2 + (c >> 4);
-          if ((c & 15) != 0) mx[k] = fmaxf(mx[k], __uint_as_float(sr[q][c]));
-        }
+        for (int c = 1; c < 15; c += 2)
+          mx[k] = fmax3(mx[k], __uint_as_float(v[c]), __uint_as_float(v[c + 1]));
+        mx[k] = fmaxf(mx[k], __uint_as_float(v[15]));
+      }
       const float m_tile =
-          fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+          fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * sl2;
+      if (tr) FA_TRACE_MARK(1 + t, it, 2);
       // raise the reference maximum only when this tile exceeds it by > 2^8
       const bool raise = m_tile > m_ref + kRescaleThreshold;
       float alpha = 1.f;
@@ -329,48 +389,63 @@ __global__ void __launch_bounds__(kThreads, 1)
         alpha = ex2_approx(m_ref - m_tile);  // 0 while m_ref is -inf
         m_ref = m_tile;
       }
+      if (it > 0 && __any_sync(0xffffffffu, raise)) {
+        // O_t holds the product through the previous tile (that MMA finished
+        // before S_t of this tile was committed): rescale it in place before
+        // the first half of P releases this tile's PV product.
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t o[16];
+          tmem_ld16(tO + c * 16, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+          tmem_st16(tO + c * 16, o);
+        }
+      }
       const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-      float ps[4] = {0.f, 0.f, 0.f, 0.f};
-      // p = 2^(x - m) as bf16 pairs, written over the first 64 columns of
-      // S_t in two halves so that only 32 packed registers are live at once.
+      const float2 sl2v = make_float2(sl2, sl2);
+      const float2 nm2 = make_float2(neg_m, neg_m);
+      float2 ps2[4];
+      // p = 2^(s * scale * log2 e - m) (the last kEmuPer32 columns of every
+      // 32 on the FMA pipe, the rest on MUFU), written as bf16 pairs over the
+      // first 64 columns of S_t in two halves of 64 keys; each half is
+      // published on its own barrier p_half[2t+h] as soon as it is in TMEM.
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pk[32];
 #pragma unroll
         for (int qq = 0; qq < 2; ++qq) {
           const int q = 2 * h + qq;
+          ps2[q] = make_float2(0.f, 0.f);
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[q][c]), sl2, neg_m));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(sr[q][c + 1]), sl2, neg_m));
-            ps[q] += p0 + p1;
-            pk[qq * 16 + (c >> 1)] = pack_bf16x2(p0, p1);
+            const float2 x = ffma2(make_float2(__uint_as_float(sr[q][c]), __uint_as_float(sr[q][c + 1])),
+                                   sl2v, nm2);
+            float2 pv;
+            if (c >= 32 - kEmuPer32) {
+              pv = exp2_poly2(x);
+            } else {
+              pv.x = ex2_approx(x.x);
+              pv.y = ex2_approx(x.y);
+            }
+            ps2[q] = fadd2(ps2[q], pv);
+            pk[qq * 16 + (c >> 1)] = pack_bf16x2(pv.x, pv.y);
           }
         }
         tmem_st32(tS + h * 32, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_half[2 * t + h]);
+        if (tr && h == 0) FA_TRACE_MARK(1 + t, it, 3);
       }
-      l_sum = l_sum * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-      if (it > 0 && __any_sync(0xffffffffu, raise)) {
-        // O_t holds the product through the previous tile (that MMA finished
-        // before S_t of this tile was committed): rescale it in place, after
-        // the scores have left the registers.
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-          tmem_st32(tO + c * 32, o);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&p_full[t]);
+      const float2 psum = fadd2(fadd2(ps2[0], ps2[1]), fadd2(ps2[2], ps2[3]));
+      l_sum = l_sum * alpha + (psum.x + psum.y);
+      if (tr) FA_TRACE_MARK(1 + t, it, 4);
     }
 
     // ------------------------------------------------------------ epilogue
-    if (ok) ok = mbar_wait(&o_full[t], 0, abort_flag, status, tmo);
+    if (ok) ok = mbar_wait(&o_full[t], 0, abort_flag, status, tmo, kSiteO);
     const bool failed = named_bar_or(1 + t, kBM, !ok);
     if (!failed) {
       tc_fence_after();
@@ -521,6 +596,13 @@ const char* fa_status_string(fa_status s) {
 
 const char* fa_last_cuda_error(void) { return fa::g_last_cuda_error; }
 
+#ifdef FA_TRACE
+// Trace builds only: device buffer of kTraceCtas*4*kTraceIters*8 uint64 (or NULL).
+int fa_trace_set(void* device_buffer) {
+  return cudaMemcpyToSymbol(fa::g_trace, &device_buffer, sizeof(device_buffer)) == cudaSuccess ? 0 : 1;
+}
+#endif
+
 void fa_set_debug(unsigned int flags, unsigned long long timeout_ns) {
   fa::g_debug_flags = flags;
   fa::g_timeout_ns = timeout_ns;
@@ -578,6 +660,13 @@ fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
   prm.N = N;
   prm.n_qblk = static_cast<int>(n_qblk);
   prm.n_kv = (N + kBN - 1) / kBN;
+  prm.BH = static_cast<int>(BH);
+  {
+    // keep the K/V of one group of heads (4*N*d bytes per head) within ~48 MB of L2
+    const long long per_head = 4ll * N * d;
+    long long g = (48ll << 20) / per_head;
+    prm.group_heads = static_cast<int>(g < 1 ? 1 : (g > BH ? BH : g));
+  }
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
   prm.timeout_ns = g_timeout_ns ? g_timeout_ns : kDefaultTimeoutNs;
   prm.debug = g_debug_flags;
@@ -591,13 +680,15 @@ fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
                 : launch<64, false>(mq, mk, mv, mo, prm, bh, st, *dev);
 }
 
-fa_status fa_get_device_status(void* stream) {
+fa_status fa_get_device_status_word(void* stream, unsigned int* word) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (word) *word = 0;
   cudaError_t e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return fa::cuda_fail(e, "cudaStreamSynchronize");
   uint32_t v = 0;
   e = cudaMemcpyFromSymbol(&v, fa::g_device_status, sizeof(v));
   if (e != cudaSuccess) return fa::cuda_fail(e, "cudaMemcpyFromSymbol");
+  if (word) *word = v;
   if (v != 0) {
     const uint32_t zero = 0;
     e = cudaMemcpyToSymbol(fa::g_device_status, &zero, sizeof(zero));
@@ -606,5 +697,7 @@ fa_status fa_get_device_status(void* stream) {
   }
   return FA_OK;
 }
+
+fa_status fa_get_device_status(void* stream) { return fa_get_device_status_word(stream, nullptr); }
 
 }  // extern "C"

@@ -63,10 +63,11 @@ enum : uint32_t {
 
 // Wait until the phase with the given parity has completed.  Gives up (and
 // returns false) when *abort is set by another thread, or after timeout_ns of
-// global time, in which case it sets *abort itself and raises the timeout bit
-// in *status.  Never traps.
+// global time, in which case it sets *abort itself and raises, in *status,
+// the timeout bit and bit 8 + site (site < 24 names the wait that gave up).
+// Never traps.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint32_t* status, uint64_t timeout_ns) {
+                                          uint32_t* status, uint64_t timeout_ns, uint32_t site) {
   const uint32_t a = smem_addr(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = global_timer_ns();
@@ -76,7 +77,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       if (*abort) return false;
       if (global_timer_ns() - t0 > timeout_ns) {
         *abort = 1;
-        if (status) atomicOr(status, kStatusTimeout);
+        if (status) atomicOr(status, kStatusTimeout | (1u << (8 + (site & 15u))));
         return false;
       }
     }
@@ -212,6 +213,26 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -291,6 +312,61 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed pairs of fp32 (one f32x2 instruction per pair).
+__device__ __forceinline__ uint64_t f2_bits(float2 a) {
+  uint64_t u;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(u) : "f"(a.x), "f"(a.y));
+  return u;
+}
+__device__ __forceinline__ float2 bits_f2(uint64_t u) {
+  float2 a;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a.x), "=f"(a.y) : "l"(u));
+  return a;
+}
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+  return bits_f2(d);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(d);
+}
+
+// 2^x on the FMA pipe, for x <= 64: 2^x = 2^j 2^f with j = round(x),
+// f = x - j in [-1/2, 1/2], 2^f from a degree-3 polynomial of minimax
+// relative error 7.5e-5 (coefficients from csrc/fit_exp2.py), and 2^j added
+// into the exponent field.  Inputs below -126 (including -inf) are clamped,
+// giving a value below 2^-126 instead of 0.
+constexpr float kExp2C0 = 0.999928057f;
+constexpr float kExp2C1 = 0.693260968f;
+constexpr float kExp2C2 = 0.242610931f;
+constexpr float kExp2C3 = 0.0551714934f;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 t = fadd2(x, make_float2(kRoundMagic, kRoundMagic));  // j in the low mantissa bits
+  const float2 j = fadd2(t, make_float2(-kRoundMagic, -kRoundMagic));
+  const float2 f = fadd2(x, make_float2(-j.x, -j.y));
+  float2 p = ffma2(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
+  p = ffma2(p, f, make_float2(kExp2C1, kExp2C1));
+  p = ffma2(p, f, make_float2(kExp2C0, kExp2C0));
+  // (bits(t) << 23) == j << 23 modulo 2^32: the exponent increment
+  const uint32_t ex = __float_as_uint(p.x) + (__float_as_uint(t.x) << 23);
+  const uint32_t ey = __float_as_uint(p.y) + (__float_as_uint(t.y) << 23);
+  return make_float2(__uint_as_float(ex), __uint_as_float(ey));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

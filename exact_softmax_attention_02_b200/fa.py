@@ -53,6 +53,8 @@ def _load():
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_get_device_status.argtypes = [vp]
     lib.fa_get_device_status.restype = c_int
+    lib.fa_get_device_status_word.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
+    lib.fa_get_device_status_word.restype = c_int
     lib.fa_last_cuda_error.argtypes = []
     lib.fa_last_cuda_error.restype = ctypes.c_char_p
     lib.fa_set_debug.argtypes = [ctypes.c_uint, ctypes.c_ulonglong]
@@ -157,6 +159,14 @@ def attention_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
 def device_status(stream=None) -> int:
     """Synchronise the stream and read-and-clear the library's device status."""
     return _load().fa_get_device_status(_stream_handle(stream))
+
+
+def device_status_word(stream=None) -> int:
+    """Synchronise, read and clear the raw device status word (0 = no failure;
+    bit 0 = a bounded wait gave up, bit 8+k = the wait at site k gave up)."""
+    w = ctypes.c_uint(0)
+    _load().fa_get_device_status_word(_stream_handle(stream), ctypes.byref(w))
+    return int(w.value)
 
 
 def set_debug(flags: int = 0, timeout_ns: int = 0) -> None:

@@ -81,6 +81,13 @@ const char* fa_status_string(fa_status status);
  */
 fa_status fa_get_device_status(void* stream);
 
+/*
+ * fa_get_device_status_word -- as fa_get_device_status, and also stores the
+ * raw status word in *word (0 = no failure; bit 0 = a wait gave up; bit 8+k =
+ * the wait at site k gave up, for diagnosis).  word may be NULL.
+ */
+fa_status fa_get_device_status_word(void* stream, unsigned int* word);
+
 /* Message of the last CUDA error seen by this library in the calling thread
  * ("" if none).  Static thread-local storage; valid until the next call. */
 const char* fa_last_cuda_error(void);

@@ -36,7 +36,8 @@ def gpu_forward(q, k, v, causal, scale=None, with_lse=True, stream=None):
     o = torch.full_like(qd, float("nan"))  # canary: unwritten elements stay NaN
     lse = torch.full(qd.shape[:3], float("nan"), device="cuda") if with_lse else None
     fa.fa_fwd(qd, kd, vd, o, lse, scale=scale, causal=causal, stream=stream)
-    assert fa.device_status(stream) == 0
+    word = fa.device_status_word(stream)
+    assert word == 0, f"device status word {word:#x}"
     return o.cpu(), (lse.cpu() if with_lse else None)
 
 
