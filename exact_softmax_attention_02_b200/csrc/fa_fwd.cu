@@ -68,6 +68,13 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // columns (of every 32) whose exponential runs on the FMA pipe instead of MUFU
 constexpr int kEmuPer32 = FA_EMU_PER32;
 static_assert(kEmuPer32 >= 0 && kEmuPer32 <= 32 && kEmuPer32 % 2 == 0, "even count per 32");
+#ifndef FA_P_HALVES
+#define FA_P_HALVES 1
+#endif
+// 1: P_t is published once per tile; 2: in two halves of 64 keys, each on its
+// own barrier, so that the PV product can start on the first half
+constexpr int kPHalves = FA_P_HALVES;
+static_assert(kPHalves == 1 || kPHalves == 2, "P is published whole or in two halves");
 constexpr uint32_t kTmemCols = 512;
 // wait sites reported in the device status word (bit 8 + site)
 enum : uint32_t {
@@ -281,14 +288,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool last = it == n_iter - 1;
         const uint32_t ph_it = static_cast<uint32_t>(it) & 1u;
         if (!(ok = mbar_wait(&kv_full[sv], static_cast<uint32_t>(iv / S) & 1u, abort_flag, status, tmo, kSiteKvFull))) break;
-        // P_t arrives in two halves of 64 keys (p_half[2t], p_half[2t+1]): the
-        // first four K-steps of the PV product start while the softmax is
-        // still on the second half.
+        // P_t arrives whole on p_half[2t], or (kPHalves == 2) in two halves
+        // of 64 keys on p_half[2t] and p_half[2t+1], so that the first four
+        // K-steps of the PV product start while the softmax is still on the
+        // second half.
         if (!(ok = mbar_wait(&p_half[0], ph_it, abort_flag, status, tmo, kSiteP))) break;
         FA_TRACE_MARK(0, it, 0);
         tc_fence_after();
         issue_pv(0, sv, it > 0, 0);
-        if (!(ok = mbar_wait(&p_half[1], ph_it, abort_flag, status, tmo, kSiteP + 1))) break;
+        if (kPHalves == 2 &&
+            !(ok = mbar_wait(&p_half[1], ph_it, abort_flag, status, tmo, kSiteP + 1))) break;
         tc_fence_after();
         issue_pv(0, sv, true, 1);
         FA_TRACE_MARK(0, it, 1);
@@ -305,7 +314,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         FA_TRACE_MARK(0, it, 3);
         tc_fence_after();
         issue_pv(1, sv, it > 0, 0);
-        if (!(ok = mbar_wait(&p_half[3], ph_it, abort_flag, status, tmo, kSiteP + 3))) break;
+        if (kPHalves == 2 &&
+            !(ok = mbar_wait(&p_half[3], ph_it, abort_flag, status, tmo, kSiteP + 3))) break;
         tc_fence_after();
         issue_pv(1, sv, true, 1);
         FA_TRACE_MARK(0, it, 4);
@@ -409,8 +419,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       float2 ps2[4];
       // p = 2^(s * scale * log2 e - m) (the last kEmuPer32 columns of every
       // 32 on the FMA pipe, the rest on MUFU), written as bf16 pairs over the
-      // first 64 columns of S_t in two halves of 64 keys; each half is
-      // published on its own barrier p_half[2t+h] as soon as it is in TMEM.
+      // first 64 columns of S_t in two halves of 64 keys, published on
+      // p_half[2t] (whole tile) or, with kPHalves == 2, each half on its own
+      // barrier p_half[2t+h] as soon as it is in TMEM.
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pk[32];
@@ -434,9 +445,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         tmem_st32(tS + h * 32, pk);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&p_half[2 * t + h]);
+        if (kPHalves == 2 || h == 1) {
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&p_half[2 * t + (kPHalves == 2 ? h : 0)]);
+        }
         if (tr && h == 0) FA_TRACE_MARK(1 + t, it, 3);
       }
       const float2 psum = fadd2(fadd2(ps2[0], ps2[1]), fadd2(ps2[2], ps2[3]));
