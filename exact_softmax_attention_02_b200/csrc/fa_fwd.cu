@@ -79,20 +79,9 @@ constexpr uint32_t kTmemCols = 512;
 // wait sites reported in the device status word (bit 8 + site)
 enum : uint32_t {
   kSiteKvEmpty = 0, kSiteQ = 1, kSiteKvFull = 2, kSiteS = 3, kSiteP = 4,  // 4..7: p_half[0..3]
-  kSiteO = 8, kSiteDebug = 9,
+  kSiteO = 8, kSiteDebug = 9, kSiteLand = 10,
 };
 constexpr int kChunkBytes = kBM * 64 * 2;  // one 64-wide, 128-row swizzled box: 16 KB
-
-template <int D>
-struct Cfg {
-  static constexpr int kChunks = D / 64;
-  static constexpr int kTileBytes = kBM * D * 2;  // a Q, K, V or O tile
-  static constexpr int kStages = D == 128 ? 4 : 8;
-  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 4 + 2 + 1 + 1;
-  static constexpr int kSmemTiles = (kQTiles + kStages) * kTileBytes;
-  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 1024;
-  static constexpr uint32_t kColO = 256;
-};
 
 struct FwdParams {
   float* lse;           // [BH][N] or nullptr
@@ -126,64 +115,105 @@ __device__ unsigned long long* g_trace;  // [kTraceCtas][4 roles][kTraceIters][8
   } while (0)
 #endif
 
-template <int D, bool CAUSAL>
+template <int D, bool PAIR>
+struct Cfg {
+  static constexpr int kChunks = D / 64;
+  static constexpr int kQBytes = kBM * D * 2;  // one query tile (reused as O staging)
+  // one ring stage: a whole K or V tile, or (PAIR) this CTA's half of one
+  static constexpr int kStageBytes = PAIR ? kBM * D : kBM * D * 2;
+  static constexpr int kKRows = PAIR ? kBN / 2 : kBN;  // key rows of a K stage
+  static constexpr int kKChunkBytes = kKRows * 128;    // one 64-wide d chunk of a K stage
+  static constexpr int kStages = (PAIR || D == 64) ? 8 : 4;
+  static constexpr int kRowsPerTile = PAIR ? 2 * kBM : kBM;  // rows of one (pair) MMA tile
+  static constexpr int kNumBars = 2 + 2 + 3 * kStages + 2 + 4 + 2 + 1 + 1;
+  static constexpr int kSmemTiles = kQTiles * kQBytes + kStages * kStageBytes;
+  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 1024;
+  static constexpr uint32_t kColO = 256;
+};
+
+// One kernel for both CTA shapes.  PAIR == false: one CTA owns two 128-row
+// query tiles and issues M=128 MMAs.  PAIR == true (d = 128): a cluster of
+// two CTAs owns two 256-row tiles; tile t of CTA r is rows 256t + 128r of the
+// pair's 512; the even CTA issues M=256 MMAs whose B operand (K for S, V for
+// PV) is split between the two CTAs' shared memory -- keys 64r..64r+63 of each
+// K tile and d columns 64r..64r+63 of each V tile -- so each CTA reads half of
+// B and loads half of every K/V tile.  Each CTA's TMA signals a local barrier;
+// a forwarding warp then arrives on the even CTA's barrier, so that both CTAs
+// can drain their own copies exactly if they have to unwind.
+template <int D, bool CAUSAL, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const FwdParams p) {
-  using C = Cfg<D>;
+  using C = Cfg<D, PAIR>;
   constexpr int S = C::kStages;
-  constexpr int TB = C::kTileBytes;
+  constexpr int QB = C::kQBytes;
+  constexpr int SB = C::kStageBytes;
+  static_assert(!PAIR || D == 128, "the pair kernel splits d = 128 into two 64-wide halves");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem;                  // kQTiles tiles (reused as O staging)
-  uint8_t* sKV = smem + kQTiles * TB;  // S stages
+  uint8_t* sQ = smem;                  // kQTiles query tiles (reused as O staging)
+  uint8_t* sKV = smem + kQTiles * QB;  // S ring stages
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemTiles);
-  uint64_t* q_full = bars;            // [2]   TMA -> MMA
-  uint64_t* kv_full = bars + 2;       // [S]   TMA -> MMA
-  uint64_t* kv_empty = kv_full + S;   // [S]   MMA -> TMA
-  uint64_t* s_full = kv_empty + S;    // [2]   MMA -> softmax
-  uint64_t* p_half = s_full + 2;      // [4]   softmax -> MMA, [2t+h] = half h of P_t (128 arrivals)
-  uint64_t* o_full = p_half + 4;      // [2]   MMA -> epilogue
-  uint64_t* mma_done = o_full + 2;    // [1]   MMA -> itself, before TMEM release
-  uint64_t* never = mma_done + 1;     // [1]   debug: nothing arrives here
+  uint64_t* q_land = bars;            // [2] own Q copies landed (PAIR; else alias of q_full)
+  uint64_t* q_full = bars + 2;        // [2] Q tile ready for the MMA
+  uint64_t* kv_land = q_full + 2;     // [S] own K/V copies landed (PAIR; else alias of kv_full)
+  uint64_t* kv_full = kv_land + S;    // [S] K/V stage ready for the MMA
+  uint64_t* kv_empty = kv_full + S;   // [S] MMA -> producers
+  uint64_t* s_full = kv_empty + S;    // [2] MMA -> softmax
+  uint64_t* p_half = s_full + 2;      // [4] softmax -> MMA, [2t+h]
+  uint64_t* o_full = p_half + 4;      // [2] MMA -> epilogue
+  uint64_t* mma_done = o_full + 2;    // [1] MMA -> itself, before TMEM release
+  uint64_t* never = mma_done + 1;     // [1] debug: nothing arrives here
+  if (!PAIR) {
+    q_land = q_full;
+    kv_land = kv_full;
+  }
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* status = &g_device_status;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // CTA order: heads in groups of p.group_heads; inside a group, query
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  // Work order: heads in groups of p.group_heads; inside a group, query
   // blocks from the heaviest (last rows: most keys when causal) to the
-  // lightest, cycling over the group's heads.  CTAs that run together then
+  // lightest, cycling over the group's heads.  Blocks that run together then
   // share the K/V of a few heads in L2, and light blocks end the grid.
   const int per_group = p.group_heads * p.n_qblk;
-  const int grp = static_cast<int>(blockIdx.x) / per_group;
-  const int rem = static_cast<int>(blockIdx.x) % per_group;
+  const int grp = unit / per_group;
+  const int rem = unit % per_group;
   const int grp_heads = min(p.group_heads, p.BH - grp * p.group_heads);
   const int bh = grp * p.group_heads + rem % grp_heads;
   const int qblk = p.n_qblk - 1 - rem / grp_heads;
-  const int q0 = qblk * kQTiles * kBM;
-  int kv_end = p.n_kv;
-  if (CAUSAL) kv_end = min(p.n_kv, (min(q0 + kQTiles * kBM, p.N) - 1) / kBN + 1);
-  const int n_iter = kv_end;  // KV tiles visited, from kv_end-1 down to 0
+  const int q0 = qblk * kQTiles * C::kRowsPerTile;  // first row of the block
+  // last key tile each query tile needs (the causal diagonal, or the end)
+  int j_last[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t)
+    j_last[t] = CAUSAL ? min(q0 + (t + 1) * C::kRowsPerTile - 1, p.N - 1) / kBN : p.n_kv - 1;
+  const int kv_end = j_last[1] + 1;
+  const int n_iter = kv_end;  // key tiles visited, from kv_end-1 down to 0
+  // iterations before a query tile's first unmasked key tile are skipped for it
+  const int first_it[2] = {kv_end - 1 - j_last[0], 0};
   const uint64_t tmo = p.timeout_ns;
 
   if (threadIdx.x == 0) {
-    mbar_init(&q_full[0], 1);
-    mbar_init(&q_full[1], 1);
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
-    }
     for (int t = 0; t < 2; ++t) {
+      if (PAIR) mbar_init(&q_land[t], 1);
+      mbar_init(&q_full[t], PAIR ? 2 : 1);
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_half[2 * t], kBM);
-      mbar_init(&p_half[2 * t + 1], kBM);
       mbar_init(&o_full[t], 1);
     }
+    for (int s = 0; s < S; ++s) {
+      if (PAIR) mbar_init(&kv_land[s], 1);
+      mbar_init(&kv_full[s], PAIR ? 2 : 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int h = 0; h < 4; ++h) mbar_init(&p_half[h], PAIR ? 2 * (kBM / 32) : kBM);
     mbar_init(mma_done, 1);
     mbar_init(never, 1);
     *abort_flag = 0;
@@ -194,169 +224,231 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmO);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(tmem_slot, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR)
+    cluster_sync();
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+
+  // rows of this CTA's query tile t
+  auto tile_row0 = [&](int t) { return q0 + t * C::kRowsPerTile + (PAIR ? static_cast<int>(rank) * kBM : 0); };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       bool ok = true;
-      mbar_arrive_expect_tx(&q_full[0], TB);
+      mbar_arrive_expect_tx(&q_land[0], QB);
       for (int c = 0; c < C::kChunks; ++c)
-        tma_load_3d(sQ + c * kChunkBytes, &tmQ, &q_full[0], c * 64, q0, bh);
+        tma_load_3d(sQ + c * kChunkBytes, &tmQ, &q_land[0], c * 64, tile_row0(0), bh);
       int i = 0;  // loads issued into the ring, in consumption order K0 V0 K1 V1 ...
       for (int it = 0; it < n_iter && ok; ++it) {
         const int j = kv_end - 1 - it;
         for (int kv = 0; kv < 2; ++kv) {
           const int s = i % S;
           const uint32_t ph = static_cast<uint32_t>(i / S) & 1u;
-          ok = mbar_wait(&kv_empty[s], ph ^ 1u, abort_flag, status, tmo, kSiteKvEmpty);
+          ok = mbar_wait<PAIR>(&kv_empty[s], ph ^ 1u, abort_flag, status, tmo, kSiteKvEmpty);
           if (!ok) break;
-          mbar_arrive_expect_tx(&kv_full[s], TB);
-          const CUtensorMap* m = kv == 0 ? &tmK : &tmV;
-          for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(sKV + s * TB + c * kChunkBytes, m, &kv_full[s], c * 64, j * kBN, bh);
+          mbar_arrive_expect_tx(&kv_land[s], SB);
+          uint8_t* st = sKV + s * SB;
+          if (kv == 0) {
+            for (int c = 0; c < C::kChunks; ++c)
+              tma_load_3d(st + c * C::kKChunkBytes, &tmK, &kv_land[s], c * 64,
+                          j * kBN + static_cast<int>(rank) * C::kKRows, bh);
+          } else if (PAIR) {
+            tma_load_3d(st, &tmV, &kv_land[s], static_cast<int>(rank) * 64, j * kBN, bh);
+          } else {
+            for (int c = 0; c < C::kChunks; ++c)
+              tma_load_3d(st + c * kChunkBytes, &tmV, &kv_land[s], c * 64, j * kBN, bh);
+          }
           ++i;
           if (it == 0 && kv == 0) {
-            mbar_arrive_expect_tx(&q_full[1], TB);
+            mbar_arrive_expect_tx(&q_land[1], QB);
             for (int c = 0; c < C::kChunks; ++c)
-              tma_load_3d(sQ + TB + c * kChunkBytes, &tmQ, &q_full[1], c * 64, q0 + kBM, bh);
+              tma_load_3d(sQ + QB + c * kChunkBytes, &tmQ, &q_land[1], c * 64, tile_row0(1), bh);
           }
         }
       }
       if (!ok) {
-        // Unwinding: wait for every copy already issued, so that none lands
+        // Unwinding: wait for every copy this CTA issued, so that none lands
         // in shared memory after the CTA has ended.
         for (int s = 0; s < S && s < i; ++s) {
           const int last = s + ((i - 1 - s) / S) * S;
-          mbar_wait_drain(&kv_full[s], static_cast<uint32_t>(last / S) & 1u, tmo);
+          mbar_wait_drain<PAIR>(&kv_land[s], static_cast<uint32_t>(last / S) & 1u, tmo);
         }
-        mbar_wait_drain(&q_full[0], 0, tmo);
-        if (i > 0) mbar_wait_drain(&q_full[1], 0, tmo);
+        mbar_wait_drain<PAIR>(&q_land[0], 0, tmo);
+        if (i > 0) mbar_wait_drain<PAIR>(&q_land[1], 0, tmo);
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ forwarder (PAIR)
+    // Each copy of this CTA that lands is announced on the even CTA's
+    // barrier, in the producer's issue order: Q0, K0, Q1, V0, K1, V1, ...
+    if (PAIR && lane == 0) {
+      auto fwd = [&](uint64_t* land, uint64_t* full, uint32_t parity) {
+        if (!mbar_wait<PAIR>(land, parity, abort_flag, status, tmo, kSiteLand)) return false;
+        mbar_arrive_cluster(mapa_shared(smem_addr(full), 0));
+        return true;
+      };
+      bool ok = fwd(&q_land[0], &q_full[0], 0);
+      for (int i = 0; i < 2 * n_iter && ok; ++i) {
+        const int s = i % S;
+        ok = fwd(&kv_land[s], &kv_full[s], static_cast<uint32_t>(i / S) & 1u);
+        if (ok && i == 0) ok = fwd(&q_land[1], &q_full[1], 0);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(kBM, kBN, false);
-      constexpr uint32_t idO = idesc_bf16_f32(kBM, D, true);
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t kM = PAIR ? 2 * kBM : kBM;
+      constexpr uint32_t idS = idesc_bf16_f32(kM, kBN, false);
+      constexpr uint32_t idO = idesc_bf16_f32(kM, D, true);
       const uint32_t sq = smem_addr(sQ);
       const uint32_t skv = smem_addr(sKV);
-      // S_t = Q_t K^T: A = Q_t (K-major), B = K tile (K-major); 16 columns of
+      // S_t = Q_t K^T: A = Q_t (K-major), B = K stage (K-major); 16 columns of
       // d per instruction, 32 bytes apart inside each 128-byte swizzled row.
       auto issue_s = [&](int t, int s) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-          const uint64_t ad = sw128_desc(sq + t * TB + off, 16, 1024);
-          const uint64_t bd = sw128_desc(skv + s * TB + off, 16, 1024);
-          mma_ss(tmem + t * kBN, ad, bd, idS, kk > 0 ? 1u : 0u);
+          const uint64_t ad = sw128_desc(sq + t * QB + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd =
+              sw128_desc(skv + s * SB + (kk >> 2) * C::kKChunkBytes + (kk & 3) * 32, 16, 1024);
+          if (PAIR)
+            mma_ss_pair(tmem + t * kBN, ad, bd, idS, kk > 0 ? 1u : 0u);
+          else
+            mma_ss(tmem + t * kBN, ad, bd, idS, kk > 0 ? 1u : 0u);
         }
       };
-      // O_t (+)= P_t V: A = P_t in TMEM (8 columns per 16 keys), B = V tile
+      // O_t (+)= P_t V: A = P_t in TMEM (8 columns per 16 keys), B = V stage
       // stored d-contiguous (MN-major): 16 keys = 2 KB apart, d halves 16 KB apart.
       auto issue_pv = [&](int t, int s, bool accumulate, int half) {
 #pragma unroll
         for (int kk = half * (kBN / 32); kk < (half + 1) * (kBN / 32); ++kk) {
-          const uint64_t bd = sw128_desc(skv + s * TB + kk * 2048, kChunkBytes, 1024);
-          mma_ts(tmem + C::kColO + t * D, tmem + t * kBN + kk * 8, bd, idO,
-                 (accumulate || kk > 0) ? 1u : 0u);
+          const uint64_t bd = sw128_desc(skv + s * SB + kk * 2048, kChunkBytes, 1024);
+          const uint32_t acc = (accumulate || kk > 0) ? 1u : 0u;
+          if (PAIR)
+            mma_ts_pair(tmem + C::kColO + t * D, tmem + t * kBN + kk * 8, bd, idO, acc);
+          else
+            mma_ts(tmem + C::kColO + t * D, tmem + t * kBN + kk * 8, bd, idO, acc);
         }
       };
-      bool ok = mbar_wait(&q_full[0], 0, abort_flag, status, tmo, kSiteQ) &&
-                mbar_wait(&kv_full[0], 0, abort_flag, status, tmo, kSiteKvFull);
-      if (ok) {
+      auto commit = [&](uint64_t* bar) {
+        if (PAIR)
+          mma_commit_pair_mc(bar, 0x3);
+        else
+          mma_commit(bar);
+      };
+      bool ok = mbar_wait<PAIR>(&kv_full[0], 0, abort_flag, status, tmo, kSiteKvFull);
+      bool q_ready[2] = {false, false};
+      for (int t = 0; t < 2 && ok; ++t) {
+        if (first_it[t] != 0) continue;
+        ok = mbar_wait<PAIR>(&q_full[t], 0, abort_flag, status, tmo, kSiteQ);
+        if (!ok) break;
+        q_ready[t] = true;
         tc_fence_after();
-        issue_s(0, 0);
-        mma_commit(&s_full[0]);
-        ok = mbar_wait(&q_full[1], 0, abort_flag, status, tmo, kSiteQ);
+        issue_s(t, 0);
+        commit(&s_full[t]);
       }
-      if (ok) {
-        tc_fence_after();
-        issue_s(1, 0);
-        mma_commit(&s_full[1]);
-        mma_commit(&kv_empty[0]);
-      }
+      if (ok) commit(&kv_empty[0]);
       for (int it = 0; it < n_iter && ok; ++it) {
         const int iv = 2 * it + 1, ik = 2 * it + 2;
         const int sv = iv % S, sk = ik % S;
         const bool last = it == n_iter - 1;
-        const uint32_t ph_it = static_cast<uint32_t>(it) & 1u;
-        if (!(ok = mbar_wait(&kv_full[sv], static_cast<uint32_t>(iv / S) & 1u, abort_flag, status, tmo, kSiteKvFull))) break;
-        // P_t arrives whole on p_half[2t], or (kPHalves == 2) in two halves
-        // of 64 keys on p_half[2t] and p_half[2t+1], so that the first four
-        // K-steps of the PV product start while the softmax is still on the
-        // second half.
-        if (!(ok = mbar_wait(&p_half[0], ph_it, abort_flag, status, tmo, kSiteP))) break;
-        FA_TRACE_MARK(0, it, 0);
-        tc_fence_after();
-        issue_pv(0, sv, it > 0, 0);
-        if (kPHalves == 2 &&
-            !(ok = mbar_wait(&p_half[1], ph_it, abort_flag, status, tmo, kSiteP + 1))) break;
-        tc_fence_after();
-        issue_pv(0, sv, true, 1);
-        FA_TRACE_MARK(0, it, 1);
-        if (last) {
-          mma_commit(&o_full[0]);
-        } else {
-          if (!(ok = mbar_wait(&kv_full[sk], static_cast<uint32_t>(ik / S) & 1u, abort_flag, status, tmo, kSiteKvFull))) break;
-          tc_fence_after();
-          issue_s(0, sk);
-          mma_commit(&s_full[0]);
-          FA_TRACE_MARK(0, it, 2);
+        if (!(ok = mbar_wait<PAIR>(&kv_full[sv], static_cast<uint32_t>(iv / S) & 1u, abort_flag, status, tmo, kSiteKvFull))) break;
+        bool k_ready = false;
+        for (int t = 0; t < 2; ++t) {
+          if (it >= first_it[t]) {
+            // P_t arrives whole on p_half[2t], or (kPHalves == 2) in two
+            // halves of 64 keys on p_half[2t] and p_half[2t+1], so that the
+            // first four K-steps of the PV product start while the softmax
+            // is still on the second half.
+            const uint32_t ph = static_cast<uint32_t>(it - first_it[t]) & 1u;
+            const bool acc = it > first_it[t];
+            if (!(ok = mbar_wait<PAIR>(&p_half[2 * t], ph, abort_flag, status, tmo, kSiteP + 2 * t))) break;
+            FA_TRACE_MARK(0, it, 3 * t);
+            tc_fence_after();
+            issue_pv(t, sv, acc, 0);
+            if (kPHalves == 2 &&
+                !(ok = mbar_wait<PAIR>(&p_half[2 * t + 1], ph, abort_flag, status, tmo, kSiteP + 2 * t + 1))) break;
+            tc_fence_after();
+            issue_pv(t, sv, true, 1);
+            FA_TRACE_MARK(0, it, 3 * t + 1);
+            if (last) commit(&o_full[t]);
+          }
+          if (!last && it + 1 >= first_it[t]) {
+            if (!k_ready) {
+              if (!(ok = mbar_wait<PAIR>(&kv_full[sk], static_cast<uint32_t>(ik / S) & 1u, abort_flag, status, tmo, kSiteKvFull))) break;
+              k_ready = true;
+            }
+            if (!q_ready[t]) {
+              if (!(ok = mbar_wait<PAIR>(&q_full[t], 0, abort_flag, status, tmo, kSiteQ))) break;
+              q_ready[t] = true;
+            }
+            tc_fence_after();
+            issue_s(t, sk);
+            commit(&s_full[t]);
+            FA_TRACE_MARK(0, it, 3 * t + 2);
+          }
         }
-        if (!(ok = mbar_wait(&p_half[2], ph_it, abort_flag, status, tmo, kSiteP + 2))) break;
-        FA_TRACE_MARK(0, it, 3);
-        tc_fence_after();
-        issue_pv(1, sv, it > 0, 0);
-        if (kPHalves == 2 &&
-            !(ok = mbar_wait(&p_half[3], ph_it, abort_flag, status, tmo, kSiteP + 3))) break;
-        tc_fence_after();
-        issue_pv(1, sv, true, 1);
-        FA_TRACE_MARK(0, it, 4);
-        mma_commit(&kv_empty[sv]);
-        if (last) {
-          mma_commit(&o_full[1]);
-        } else {
-          issue_s(1, sk);
-          mma_commit(&s_full[1]);
-          mma_commit(&kv_empty[sk]);
-          FA_TRACE_MARK(0, it, 5);
-        }
+        if (!ok) break;
+        commit(&kv_empty[sv]);
+        if (!last) commit(&kv_empty[sk]);
       }
       // every MMA issued here has finished before TMEM is released
-      mma_commit(mma_done);
-      mbar_wait_drain(mma_done, 0, tmo);
+      if (PAIR)
+        mma_commit_pair_mc(mma_done, 0x1);
+      else
+        mma_commit(mma_done);
+      mbar_wait_drain<PAIR>(mma_done, 0, tmo);
     }
   } else if (warp >= kSoftmaxWarp0) {
     // ------------------------------------------------------------ softmax
     const int t = (warp - kSoftmaxWarp0) >> 2;  // query tile of this warpgroup
     const int wq = warp & 3;                    // TMEM lane quarter
     const int r = wq * 32 + lane;               // row inside the tile
-    const int row = q0 + t * kBM + r;           // query index in the head
+    const int row0 = tile_row0(t);
+    const int row = row0 + r;                   // query index in the head
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_base + t * kBN;
     const uint32_t tO = tmem + lane_base + C::kColO + t * D;
     const float sl2 = p.scale_log2;
-    const int tile_first_row = q0 + t * kBM;
     // last key this row may see
     const int key_limit = CAUSAL ? min(row, p.N - 1) : p.N - 1;
+    // O_t holds the product through the previous tile (that MMA finished
+    // before S_t of this tile was committed): rescale this thread's row of
+    // it in place, before P of this tile releases the next PV product.
+    auto rescale_o_rows = [&](uint32_t taddr, float a) {
+#pragma unroll
+      for (int c = 0; c < D / 16; ++c) {
+        uint32_t o[16];
+        tmem_ld16(taddr + c * 16, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * a);
+        tmem_st16(taddr + c * 16, o);
+      }
+    };
 
     float m_ref = -INFINITY;  // reference maximum, log2 units of scaled scores
     float l_sum = 0.f;        // running denominator relative to m_ref
     bool ok = true;
     if (p.debug & 1u) {
-      ok = __all_sync(0xffffffffu, mbar_wait(never, 0, abort_flag, status, tmo, kSiteDebug));
+      ok = __all_sync(0xffffffffu, mbar_wait<PAIR>(never, 0, abort_flag, status, tmo, kSiteDebug));
     }
-    for (int it = 0; it < n_iter && ok; ++it) {
+    for (int it = first_it[t]; it < n_iter && ok; ++it) {
+      const int li = it - first_it[t];
       const int j = kv_end - 1 - it;
       ok = __all_sync(0xffffffffu,
-                      mbar_wait(&s_full[t], static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteS));
+                      mbar_wait<PAIR>(&s_full[t], static_cast<uint32_t>(li) & 1u, abort_flag, status, tmo, kSiteS));
       if (!ok) break;
       const bool tr = lane == 0 && (warp & 3) == 0;
       if (tr) FA_TRACE_MARK(1 + t, it, 0);
@@ -368,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tr) FA_TRACE_MARK(1 + t, it, 1);
 
       const int kbase = j * kBN;
-      const bool masked = (kbase + kBN > p.N) || (CAUSAL && kbase + kBN - 1 > tile_first_row);
+      const bool masked = (kbase + kBN > p.N) || (CAUSAL && kbase + kBN - 1 > row0);
       if (masked) {
 #pragma unroll
         for (int q = 0; q < 4; ++q)
@@ -399,20 +491,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         alpha = ex2_approx(m_ref - m_tile);  // 0 while m_ref is -inf
         m_ref = m_tile;
       }
-      if (it > 0 && __any_sync(0xffffffffu, raise)) {
-        // O_t holds the product through the previous tile (that MMA finished
-        // before S_t of this tile was committed): rescale it in place before
-        // the first half of P releases this tile's PV product.
-#pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
-          uint32_t o[16];
-          tmem_ld16(tO + c * 16, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-          tmem_st16(tO + c * 16, o);
-        }
-      }
+      const bool rescale_o = li > 0 && __any_sync(0xffffffffu, raise);
+      if (kPHalves == 2 && rescale_o) rescale_o_rows(tO, alpha);
       const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
       const float2 sl2v = make_float2(sl2, sl2);
       const float2 nm2 = make_float2(neg_m, neg_m);
@@ -445,10 +525,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         tmem_st32(tS + h * 32, pk);
+        // whole-P: the rescale waits until the scores have left the registers
+        if (kPHalves == 1 && h == 1 && rescale_o) rescale_o_rows(tO, alpha);
         if (kPHalves == 2 || h == 1) {
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(&p_half[2 * t + (kPHalves == 2 ? h : 0)]);
+          uint64_t* pbar = &p_half[2 * t + ((kPHalves == 2 && h == 1) ? 1 : 0)];
+          if (PAIR) {
+            // one arrival per warp on the even CTA's barrier, after every
+            // lane's stores are complete and fenced
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster_relaxed(mapa_shared(smem_addr(pbar), 0));
+          } else {
+            mbar_arrive(pbar);
+          }
         }
         if (tr && h == 0) FA_TRACE_MARK(1 + t, it, 3);
       }
@@ -458,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ------------------------------------------------------------ epilogue
-    if (ok) ok = mbar_wait(&o_full[t], 0, abort_flag, status, tmo, kSiteO);
+    if (ok) ok = mbar_wait<PAIR>(&o_full[t], 0, abort_flag, status, tmo, kSiteO);
     const bool failed = named_bar_or(1 + t, kBM, !ok);
     if (!failed) {
       tc_fence_after();
@@ -469,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // O_t / l -> bf16 -> the Q_t buffer (no MMA reads it any more), laid
       // out as the 128-byte-swizzled boxes the store tensor map expects.
-      uint8_t* stage = sQ + t * TB;
+      uint8_t* stage = sQ + t * QB;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -489,9 +579,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       named_bar_sync(1 + t, kBM);
-      if (r == 0 && tile_first_row < p.N) {
+      if (r == 0 && row0 < p.N) {
         for (int c = 0; c < C::kChunks; ++c)
-          tma_store_3d(&tmO, stage + c * kChunkBytes, c * 64, tile_first_row, bh);
+          tma_store_3d(&tmO, stage + c * kChunkBytes, c * 64, row0, bh);
         bulk_commit_group();
         bulk_wait_group_read0();
       }
@@ -499,11 +589,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  if (PAIR)
+    cluster_sync();
+  else
+    __syncthreads();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    if (PAIR)
+      tmem_dealloc_pair(tmem, kTmemCols);
+    else
+      tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -536,16 +632,16 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
   return fn;
 }
 
-// [BH][N][d] bf16 viewed as a 3-D tensor (d fastest); boxes of 64 x 128 x 1
-// with the 128-byte swizzle.  Rows past N read as zero and are not stored.
-bool make_map(CUtensorMap* map, const void* base, int d, int N, int BH) {
+// [BH][N][d] bf16 viewed as a 3-D tensor (d fastest); boxes of 64 x box_rows
+// x 1 with the 128-byte swizzle.  Rows past N read as zero and are not stored.
+bool make_map(CUtensorMap* map, const void* base, int d, int N, int BH, int box_rows) {
   auto enc = encode_tiled();
   if (!enc) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                         static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                            static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kBM), 1};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -556,27 +652,61 @@ bool make_map(CUtensorMap* map, const void* base, int d, int N, int BH) {
 struct DeviceInfo {
   bool checked = false;
   bool sm100 = false;
-  bool attr_set[4] = {false, false, false, false};
+  bool attr_set[8] = {};
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_devices[kMaxDevices];
 std::mutex g_dev_mutex;
 
+// The pair kernel (clusters of two CTAs, M = 256 MMAs) is built for d = 128
+// only when FA_PAIR is defined: on B200 it measured slower than one CTA per
+// block (the two SMs' softmax steps gate every shared MMA).
+#ifdef FA_PAIR
+template <int D>
+constexpr bool kUsePair = (D == 128);
+#else
+template <int D>
+constexpr bool kUsePair = false;
+#endif
+
 template <int D, bool CAUSAL>
-fa_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                 const CUtensorMap& mo, const FwdParams& prm, int BH, cudaStream_t stream,
-                 DeviceInfo& dev) {
-  constexpr int slot = (D == 128 ? 2 : 0) + (CAUSAL ? 1 : 0);
-  auto kern = fa_fwd_kernel<D, CAUSAL>;
+fa_status launch(const void* Q, const void* K, const void* V, void* O, FwdParams prm, int N, int BH,
+                 cudaStream_t stream, DeviceInfo& dev) {
+  constexpr bool PAIR = kUsePair<D>;
+  using C = Cfg<D, PAIR>;
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_map(&mq, Q, D, N, BH, kBM) || !make_map(&mk, K, D, N, BH, C::kKRows) ||
+      !make_map(&mv, V, D, N, BH, kBM) || !make_map(&mo, O, D, N, BH, kBM)) {
+    snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed");
+    return FA_ERR_CUDA;
+  }
+  const long long rows_per_block = static_cast<long long>(kQTiles) * C::kRowsPerTile;
+  prm.n_qblk = static_cast<int>((N + rows_per_block - 1) / rows_per_block);
+  const long long units = static_cast<long long>(BH) * prm.n_qblk;
+  const long long grid = units * (PAIR ? 2 : 1);
+  if (grid > 0x7fffffffll) return FA_ERR_SHAPE;
+  constexpr int slot = (D == 128 ? 4 : 0) + (CAUSAL ? 2 : 0) + (PAIR ? 1 : 0);
+  auto kern = fa_fwd_kernel<D, CAUSAL, PAIR>;
   if (!dev.attr_set[slot]) {
     cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::kSmemBytes);
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
     dev.attr_set[slot] = true;
   }
-  const long long grid = static_cast<long long>(BH) * prm.n_qblk;
-  kern<<<static_cast<unsigned>(grid), kThreads, Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, mo, prm);
-  cudaError_t e = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = PAIR ? 2 : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, prm);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
   return FA_OK;
 }
@@ -662,16 +792,10 @@ fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
   }
   if (!dev->sm100) return FA_ERR_UNSUPPORTED;
 
-  CUtensorMap mq, mk, mv, mo;
-  if (!make_map(&mq, Q, d, N, static_cast<int>(BH)) || !make_map(&mk, K, d, N, static_cast<int>(BH)) ||
-      !make_map(&mv, V, d, N, static_cast<int>(BH)) || !make_map(&mo, O, d, N, static_cast<int>(BH))) {
-    snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed");
-    return FA_ERR_CUDA;
-  }
   FwdParams prm;
   prm.lse = LSE;
   prm.N = N;
-  prm.n_qblk = static_cast<int>(n_qblk);
+  prm.n_qblk = 0;  // set per kernel shape in launch()
   prm.n_kv = (N + kBN - 1) / kBN;
   prm.BH = static_cast<int>(BH);
   {
@@ -687,10 +811,10 @@ fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
   const int bh = static_cast<int>(BH);
   std::lock_guard<std::mutex> lock(g_dev_mutex);
   if (d == 128)
-    return causal ? launch<128, true>(mq, mk, mv, mo, prm, bh, st, *dev)
-                  : launch<128, false>(mq, mk, mv, mo, prm, bh, st, *dev);
-  return causal ? launch<64, true>(mq, mk, mv, mo, prm, bh, st, *dev)
-                : launch<64, false>(mq, mk, mv, mo, prm, bh, st, *dev);
+    return causal ? launch<128, true>(Q, K, V, O, prm, N, bh, st, *dev)
+                  : launch<128, false>(Q, K, V, O, prm, N, bh, st, *dev);
+  return causal ? launch<64, true>(Q, K, V, O, prm, N, bh, st, *dev)
+                : launch<64, false>(Q, K, V, O, prm, N, bh, st, *dev);
 }
 
 fa_status fa_get_device_status_word(void* stream, unsigned int* word) {
