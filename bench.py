@@ -276,7 +276,7 @@ def run_reference(args, w):
     if rank != 0:
         return 0
     q32, k32, v32 = oracle_inputs(w, w.seed)
-    budget_per_step = min(8.0, 150.0 / max(1, args.steps + args.warmup))
+    budget_per_step = min(args.ref_step_seconds, 150.0 / max(1, args.steps + args.warmup))
     n = 32
     dt, _ = oracle_sample_time(w, q32, k32, v32, random_rows(w, n, 1))
     n = int(max(8, min(w.B * w.H * w.N, n * budget_per_step / max(dt, 1e-3))))
@@ -325,8 +325,20 @@ def run_ours(args, w):
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    splits = None
+    launches_per_step = 1
+    if args.path == "splitkv":
+        splits = args.splits if args.splits > 0 else fa.splitkv_default_splits(w.B, w.H, w.N, w.d, w.causal)
+        ws = torch.empty(max(16, fa.splitkv_workspace_bytes(w.B, w.H, w.N, w.d, splits, w.causal)),
+                         dtype=torch.uint8, device=dev)
+        launches_per_step = 1 if splits == 1 else 2  # split kernel + merge
+
     def step():
-        fa.fa_fwd(q, k, v, o, lse, scale=w.scale, causal=w.causal, stream=stream)
+        if splits is None:
+            fa.fa_fwd(q, k, v, o, lse, scale=w.scale, causal=w.causal, stream=stream)
+        else:
+            fa.fa_fwd_splitkv(q, k, v, o, lse, workspace=ws, num_splits=splits, scale=w.scale,
+                              causal=w.causal, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -364,14 +376,16 @@ def run_ours(args, w):
     q_p, k_p, v_p = (t.pin_memory() for t in (q_h, k_h, v_h))
     e2e_steps = max(3, min(args.steps, 20))
     for _ in range(2):
-        fa.attention_forward(q_p, k_p, v_p, scale=w.scale, causal=w.causal, out=(o_h, lse_h))
+        fa.attention_forward(q_p, k_p, v_p, scale=w.scale, causal=w.causal, out=(o_h, lse_h),
+                             num_splits=splits)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        fa.attention_forward(q_p, k_p, v_p, scale=w.scale, causal=w.causal, out=(o_h, lse_h))
+        fa.attention_forward(q_p, k_p, v_p, scale=w.scale, causal=w.causal, out=(o_h, lse_h),
+                             num_splits=splits)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist, dev)
@@ -383,7 +397,7 @@ def run_ours(args, w):
     peak, peak_src = tensor_peak()
     achieved = w.flops / avg_launch_s / 1e12
     traffic = committed_traffic(w.name)
-    launches = int(sum_over_ranks(args.steps, dist, dev))
+    launches = int(sum_over_ranks(args.steps * launches_per_step, dist, dev))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -399,13 +413,15 @@ def run_ours(args, w):
             "ms_per_step": 1e3 * elapsed_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16 Q/K/V per rank)",
-            "config": {**w.as_config(), "parallelism": f"replicas{world}",
+            "config": {**w.as_config(), "parallelism": f"replicas{world}", "path": args.path,
+                       **({"num_splits": splits} if splits is not None else {}),
                        "l2": (f"inputs+outputs {in_bytes / 1e6:.0f} MB > L2 126 MB, no flush"
                               if in_bytes > L2_BYTES else "L2 not flushed (inputs < L2)")},
             "pct_of_peak": 100.0 * value / world / peak,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": peak_src, "kernel": f"fa_fwd_kernel<{w.d},{str(w.causal).lower()}>",
+                         "peak_source": peak_src,
+                         "kernel": f"fa_fwd_kernel<{w.d},{str(w.causal).lower()}>" + (" + fa_merge_kernel" if launches_per_step == 2 else ""),
                          "kernel_source_sha256": kernel_source_hash()},
             "e2e": {"value": weak_scaling_value(w.flops, world, e2e_steps, e2e_s), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -429,7 +445,12 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--path", default="fused", choices=["fused", "splitkv"],
+                    help="fused: fa_fwd; splitkv: fa_fwd_splitkv (key ranges + merge)")
+    ap.add_argument("--splits", type=int, default=0, help="splitkv: key ranges (0 = default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-step-seconds", type=float, default=8.0,
+                    help="reference arm: target oracle seconds per step (bounded sample)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

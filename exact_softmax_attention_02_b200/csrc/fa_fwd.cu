@@ -93,6 +93,13 @@ struct FwdParams {
   float scale_log2;     // scale * log2(e)
   uint64_t timeout_ns;  // bound on every wait
   uint32_t debug;       // bit 0: stall the softmax warps on a barrier nobody signals
+  // split-KV only: the key tiles of a query block are divided into
+  // num_splits ranges of kv_per_split tiles; each CTA writes the normalised
+  // partial output and partial LSE of its range (fp32, row-major)
+  int num_splits;
+  int kv_per_split;
+  float* o_part;    // [num_splits][BH][N][d]
+  float* lse_part;  // [num_splits][BH][N]
 };
 
 __device__ uint32_t g_device_status;
@@ -140,7 +147,7 @@ struct Cfg {
 // B and loads half of every K/V tile.  Each CTA's TMA signals a local barrier;
 // a forwarding warp then arrives on the even CTA's barrier, so that both CTAs
 // can drain their own copies exactly if they have to unwind.
-template <int D, bool CAUSAL, bool PAIR>
+template <int D, bool CAUSAL, bool PAIR, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -150,6 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int QB = C::kQBytes;
   constexpr int SB = C::kStageBytes;
   static_assert(!PAIR || D == 128, "the pair kernel splits d = 128 into two 64-wide halves");
+  static_assert(!(PAIR && SPLIT), "split-KV uses the single-CTA shape");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -178,7 +186,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
-  const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int split = SPLIT ? static_cast<int>(blockIdx.x % p.num_splits) : 0;
+  const int unit = SPLIT  ? static_cast<int>(blockIdx.x / p.num_splits)
+                   : PAIR ? static_cast<int>(blockIdx.x >> 1)
+                          : static_cast<int>(blockIdx.x);
   // Work order: heads in groups of p.group_heads; inside a group, query
   // blocks from the heaviest (last rows: most keys when causal) to the
   // lightest, cycling over the group's heads.  Blocks that run together then
@@ -195,10 +206,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
   for (int t = 0; t < 2; ++t)
     j_last[t] = CAUSAL ? min(q0 + (t + 1) * C::kRowsPerTile - 1, p.N - 1) / kBN : p.n_kv - 1;
-  const int kv_end = j_last[1] + 1;
-  const int n_iter = kv_end;  // key tiles visited, from kv_end-1 down to 0
-  // iterations before a query tile's first unmasked key tile are skipped for it
-  const int first_it[2] = {kv_end - 1 - j_last[0], 0};
+  // key tiles [kv_lo, kv_end) of this CTA (all of them unless split), visited
+  // from kv_end-1 down to kv_lo
+  const int kv_lo = SPLIT ? split * p.kv_per_split : 0;
+  const int kv_end = SPLIT ? min(j_last[1] + 1, kv_lo + p.kv_per_split) : j_last[1] + 1;
+  const int n_iter = max(0, kv_end - kv_lo);
+  // iterations before a query tile's first unmasked key tile are skipped for
+  // it; a tile whose first iteration is past n_iter has no keys in this range
+  const int first_it[2] = {kv_end - 1 - min(j_last[0], kv_end - 1), 0};
+  const bool tile_active[2] = {first_it[0] < n_iter, n_iter > 0};
   const uint64_t tmo = p.timeout_ns;
 
   if (threadIdx.x == 0) {
@@ -245,11 +261,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if (lane == 0 && n_iter > 0) {
       bool ok = true;
-      mbar_arrive_expect_tx(&q_land[0], QB);
-      for (int c = 0; c < C::kChunks; ++c)
-        tma_load_3d(sQ + c * kChunkBytes, &tmQ, &q_land[0], c * 64, tile_row0(0), bh);
+      if (tile_active[0]) {
+        mbar_arrive_expect_tx(&q_land[0], QB);
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_3d(sQ + c * kChunkBytes, &tmQ, &q_land[0], c * 64, tile_row0(0), bh);
+      }
       int i = 0;  // loads issued into the ring, in consumption order K0 V0 K1 V1 ...
       for (int it = 0; it < n_iter && ok; ++it) {
         const int j = kv_end - 1 - it;
@@ -285,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int last = s + ((i - 1 - s) / S) * S;
           mbar_wait_drain<PAIR>(&kv_land[s], static_cast<uint32_t>(last / S) & 1u, tmo);
         }
-        mbar_wait_drain<PAIR>(&q_land[0], 0, tmo);
+        if (tile_active[0]) mbar_wait_drain<PAIR>(&q_land[0], 0, tmo);
         if (i > 0) mbar_wait_drain<PAIR>(&q_land[1], 0, tmo);
       }
     }
@@ -308,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && rank == 0) {
+    if (lane == 0 && rank == 0 && n_iter > 0) {
       constexpr uint32_t kM = PAIR ? 2 * kBM : kBM;
       constexpr uint32_t idS = idesc_bf16_f32(kM, kBN, false);
       constexpr uint32_t idO = idesc_bf16_f32(kM, D, true);
@@ -548,9 +566,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ------------------------------------------------------------ epilogue
-    if (ok) ok = mbar_wait<PAIR>(&o_full[t], 0, abort_flag, status, tmo, kSiteO);
+    if (ok && tile_active[t]) ok = mbar_wait<PAIR>(&o_full[t], 0, abort_flag, status, tmo, kSiteO);
     const bool failed = named_bar_or(1 + t, kBM, !ok);
-    if (!failed) {
+    if (!failed && SPLIT) {
+      // partial state of this key range: u / l (fp32) and its LSE; a range
+      // with no allowed key for this row gives LSE = -inf and weight 0 in
+      // the merge
+      tc_fence_after();
+      const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
+      const float lse_val = l_sum > 0.f ? (m_ref + log2f(l_sum)) * 0.69314718055994530942f : -INFINITY;
+      const size_t prow = (static_cast<size_t>(split) * p.BH + bh) * p.N + row;
+      float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D);
+      if (row < p.N) p.lse_part[prow] = lse_val;
+      if (tile_active[t]) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld();
+          if (row < p.N) {
+#pragma unroll
+            for (int g = 0; g < 8; ++g)
+              dst[c * 8 + g] = make_float4(__uint_as_float(o[4 * g]) * inv_l, __uint_as_float(o[4 * g + 1]) * inv_l,
+                                           __uint_as_float(o[4 * g + 2]) * inv_l, __uint_as_float(o[4 * g + 3]) * inv_l);
+          }
+        }
+      } else if (row < p.N) {
+#pragma unroll
+        for (int g = 0; g < D / 4; ++g) dst[g] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    } else if (!failed) {
       tc_fence_after();
       const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
       if (p.lse != nullptr && row < p.N) {
@@ -603,6 +648,52 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Merge of the split-KV partial states of every row: with M = max_s LSE_s
+// and w_s = e^(LSE_s - M) (0 for an empty range), O = sum_s w_s O_s / sum_s
+// w_s and LSE = M + ln sum_s w_s -- the block update applied to whole states
+// (liminalml.com "FlashAttention", m' = max(m, max s) and the rescale of
+// both numerator and denominator; interactiveml.org, the merge with the
+// guard for m = -inf).  One warp per row; each lane owns d/32 columns.
+template <int D>
+__global__ void __launch_bounds__(256)
+    fa_merge_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
+                    __nv_bfloat16* __restrict__ O, float* __restrict__ LSE, long long rows,
+                    int num_splits) {
+  constexpr int kPer = D / 32;
+  const long long row = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float m = -INFINITY;
+  for (int s = 0; s < num_splits; ++s) m = fmaxf(m, lse_part[s * rows + row]);
+  float acc[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) acc[i] = 0.f;
+  float wsum = 0.f;
+  for (int s = 0; s < num_splits; ++s) {
+    const float l = lse_part[s * rows + row];
+    const float w = (l == -INFINITY) ? 0.f : ex2_approx((l - m) * 1.4426950408889634f);
+    wsum += w;
+    const float* src = o_part + (s * rows + row) * D + lane * kPer;
+    if (kPer == 4) {
+      const float4 v = *reinterpret_cast<const float4*>(src);
+      acc[0] += w * v.x;
+      acc[1] += w * v.y;
+      acc[2] += w * v.z;
+      acc[3] += w * v.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) acc[i] += w * src[i];
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  __nv_bfloat16* dst = O + row * D + lane * kPer;
+#pragma unroll
+  for (int i = 0; i < kPer; i += 2) {
+    *reinterpret_cast<__nv_bfloat162*>(dst + i) = __floats2bfloat162_rn(acc[i] * inv, acc[i + 1] * inv);
+  }
+  if (LSE != nullptr && lane == 0) LSE[row] = wsum > 0.f ? m + logf(wsum) : -INFINITY;
+}
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
@@ -652,7 +743,7 @@ bool make_map(CUtensorMap* map, const void* base, int d, int N, int BH, int box_
 struct DeviceInfo {
   bool checked = false;
   bool sm100 = false;
-  bool attr_set[8] = {};
+  bool attr_set[16] = {};
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_devices[kMaxDevices];
@@ -669,10 +760,10 @@ template <int D>
 constexpr bool kUsePair = false;
 #endif
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool SPLIT>
 fa_status launch(const void* Q, const void* K, const void* V, void* O, FwdParams prm, int N, int BH,
                  cudaStream_t stream, DeviceInfo& dev) {
-  constexpr bool PAIR = kUsePair<D>;
+  constexpr bool PAIR = kUsePair<D> && !SPLIT;
   using C = Cfg<D, PAIR>;
   CUtensorMap mq, mk, mv, mo;
   if (!make_map(&mq, Q, D, N, BH, kBM) || !make_map(&mk, K, D, N, BH, C::kKRows) ||
@@ -683,10 +774,10 @@ fa_status launch(const void* Q, const void* K, const void* V, void* O, FwdParams
   const long long rows_per_block = static_cast<long long>(kQTiles) * C::kRowsPerTile;
   prm.n_qblk = static_cast<int>((N + rows_per_block - 1) / rows_per_block);
   const long long units = static_cast<long long>(BH) * prm.n_qblk;
-  const long long grid = units * (PAIR ? 2 : 1);
+  const long long grid = units * (SPLIT ? prm.num_splits : (PAIR ? 2 : 1));
   if (grid > 0x7fffffffll) return FA_ERR_SHAPE;
-  constexpr int slot = (D == 128 ? 4 : 0) + (CAUSAL ? 2 : 0) + (PAIR ? 1 : 0);
-  auto kern = fa_fwd_kernel<D, CAUSAL, PAIR>;
+  constexpr int slot = (D == 128 ? 8 : 0) + (CAUSAL ? 4 : 0) + (PAIR ? 2 : 0) + (SPLIT ? 1 : 0);
+  auto kern = fa_fwd_kernel<D, CAUSAL, PAIR, SPLIT>;
   if (!dev.attr_set[slot]) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -711,6 +802,19 @@ fa_status launch(const void* Q, const void* K, const void* V, void* O, FwdParams
   return FA_OK;
 }
 
+template <int D>
+fa_status launch_merge(const float* o_part, const float* lse_part, void* O, float* LSE, long long rows,
+                       int num_splits, cudaStream_t stream) {
+  constexpr int kWarps = 8;
+  const long long blocks = (rows + kWarps - 1) / kWarps;
+  if (blocks > 0x7fffffffll) return FA_ERR_SHAPE;
+  fa_merge_kernel<D><<<static_cast<unsigned>(blocks), kWarps * 32, 0, stream>>>(
+      o_part, lse_part, static_cast<__nv_bfloat16*>(O), LSE, rows, num_splits);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  return FA_OK;
+}
+
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
   return x < y + nb && y < x + na;
@@ -732,7 +836,8 @@ const char* fa_status_string(fa_status s) {
     case FA_ERR_ALIGN: return "FA_ERR_ALIGN: Q/K/V/O need 16-byte, LSE 4-byte alignment";
     case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA call or kernel launch failed";
     case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT: a kernel gave up on a bounded wait";
-    case FA_ERR_ALIAS: return "FA_ERR_ALIAS: O or LSE overlaps an input or each other";
+    case FA_ERR_ALIAS: return "FA_ERR_ALIAS: O, LSE or the workspace overlaps an input or each other";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: the workspace is smaller than required";
   }
   return "unknown fa_status";
 }
@@ -751,9 +856,14 @@ void fa_set_debug(unsigned int flags, unsigned long long timeout_ns) {
   fa::g_timeout_ns = timeout_ns;
 }
 
-fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H,
-                 int N, int d, float scale, int causal, void* stream) {
-  using namespace fa;
+}  // extern "C"
+
+namespace fa {
+namespace {
+
+// Argument checks shared by the forward entry points (host only).
+fa_status check_args(const void* Q, const void* K, const void* V, const void* O, const float* LSE,
+                     int B, int H, int N, int d, float scale) {
   if (!Q || !K || !V || !O) return FA_ERR_NULL;
   if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
   if (!std::isfinite(scale)) return FA_ERR_SHAPE;
@@ -773,48 +883,160 @@ fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
   if (LSE && (overlaps(LSE, lbytes, Q, nbytes) || overlaps(LSE, lbytes, K, nbytes) ||
               overlaps(LSE, lbytes, V, nbytes) || overlaps(LSE, lbytes, O, nbytes)))
     return FA_ERR_ALIAS;
+  return FA_OK;
+}
 
+// After check_args: the current device must be an sm_100 GPU; fills *prm
+// (all but n_qblk and the split fields) and *dev.
+fa_status prepare(const float* LSE, int B, int H, int N, int d, float scale, FwdParams* prm,
+                  DeviceInfo** dev) {
+  const long long BH = static_cast<long long>(B) * H;
   int dev_id = 0;
   cudaError_t e = cudaGetDevice(&dev_id);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev_id < 0 || dev_id >= kMaxDevices) return FA_ERR_UNSUPPORTED;
-  DeviceInfo* dev;
   {
     std::lock_guard<std::mutex> lock(g_dev_mutex);
-    dev = &g_devices[dev_id];
-    if (!dev->checked) {
+    *dev = &g_devices[dev_id];
+    if (!(*dev)->checked) {
       int major = 0;
       e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev_id);
       if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
-      dev->sm100 = (major == 10);
-      dev->checked = true;
+      (*dev)->sm100 = (major == 10);
+      (*dev)->checked = true;
     }
   }
-  if (!dev->sm100) return FA_ERR_UNSUPPORTED;
+  if (!(*dev)->sm100) return FA_ERR_UNSUPPORTED;
 
-  FwdParams prm;
-  prm.lse = LSE;
-  prm.N = N;
-  prm.n_qblk = 0;  // set per kernel shape in launch()
-  prm.n_kv = (N + kBN - 1) / kBN;
-  prm.BH = static_cast<int>(BH);
+  *prm = FwdParams{};
+  prm->lse = const_cast<float*>(LSE);
+  prm->N = N;
+  prm->n_qblk = 0;  // set per kernel shape in launch()
+  prm->n_kv = (N + kBN - 1) / kBN;
+  prm->BH = static_cast<int>(BH);
   {
     // keep the K/V of one group of heads (4*N*d bytes per head) within ~48 MB of L2
     const long long per_head = 4ll * N * d;
     long long g = (48ll << 20) / per_head;
-    prm.group_heads = static_cast<int>(g < 1 ? 1 : (g > BH ? BH : g));
+    prm->group_heads = static_cast<int>(g < 1 ? 1 : (g > BH ? BH : g));
   }
-  prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
-  prm.timeout_ns = g_timeout_ns ? g_timeout_ns : kDefaultTimeoutNs;
-  prm.debug = g_debug_flags;
+  prm->scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
+  prm->timeout_ns = g_timeout_ns ? g_timeout_ns : kDefaultTimeoutNs;
+  prm->debug = g_debug_flags;
+  prm->num_splits = 1;
+  return FA_OK;
+}
+
+constexpr int kMaxSplits = 256;
+
+long long splitkv_rows(int B, int H, int N) { return static_cast<long long>(B) * H * N; }
+
+size_t splitkv_bytes(int B, int H, int N, int d, int num_splits) {
+  const long long rows = splitkv_rows(B, H, N);
+  return static_cast<size_t>(num_splits) * static_cast<size_t>(rows) * (static_cast<size_t>(d) + 1) * 4;
+}
+
+int default_splits(int B, int H, int N, bool causal) {
+  const long long units = static_cast<long long>(B) * H * ((N + kQTiles * kBM - 1) / (kQTiles * kBM));
+  const int n_kv = (N + kBN - 1) / kBN;
+  // non-causal: as many ranges as fit in one wave of 148 SMs without starting
+  // a second; causal (uneven ranges): at least one and a half waves; at least
+  // two key tiles per range.  Chosen from measurements on B200.
+  long long s = causal ? (222 + units - 1) / units : 148 / units;
+  const long long cap = n_kv / 2 > 1 ? n_kv / 2 : 1;
+  if (s > cap) s = cap;
+  if (s > kMaxSplits) s = kMaxSplits;
+  return static_cast<int>(s < 1 ? 1 : s);
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" {
+
+fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H,
+                 int N, int d, float scale, int causal, void* stream) {
+  using namespace fa;
+  FwdParams prm;
+  DeviceInfo* dev = nullptr;
+  fa_status st0 = check_args(Q, K, V, O, LSE, B, H, N, d, scale);
+  if (st0 == FA_OK) st0 = prepare(LSE, B, H, N, d, scale, &prm, &dev);
+  if (st0 != FA_OK) return st0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int bh = static_cast<int>(BH);
+  const int bh = prm.BH;
   std::lock_guard<std::mutex> lock(g_dev_mutex);
   if (d == 128)
-    return causal ? launch<128, true>(Q, K, V, O, prm, N, bh, st, *dev)
-                  : launch<128, false>(Q, K, V, O, prm, N, bh, st, *dev);
-  return causal ? launch<64, true>(Q, K, V, O, prm, N, bh, st, *dev)
-                : launch<64, false>(Q, K, V, O, prm, N, bh, st, *dev);
+    return causal ? launch<128, true, false>(Q, K, V, O, prm, N, bh, st, *dev)
+                  : launch<128, false, false>(Q, K, V, O, prm, N, bh, st, *dev);
+  return causal ? launch<64, true, false>(Q, K, V, O, prm, N, bh, st, *dev)
+                : launch<64, false, false>(Q, K, V, O, prm, N, bh, st, *dev);
+}
+
+int fa_fwd_splitkv_default_splits(int B, int H, int N, int d, int causal) {
+  (void)d;
+  if (B < 1 || H < 1 || N < 1) return 1;
+  return fa::default_splits(B, H, N, causal != 0);
+}
+
+size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int N, int d, int causal, int num_splits) {
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  if (num_splits <= 0) num_splits = fa::default_splits(B, H, N, causal != 0);
+  if (num_splits > fa::kMaxSplits) return 0;
+  return fa::splitkv_bytes(B, H, N, d, num_splits);
+}
+
+fa_status fa_fwd_splitkv(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                         void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+                         float scale, int causal, int num_splits, void* stream) {
+  using namespace fa;
+  FwdParams prm;
+  DeviceInfo* dev = nullptr;
+  fa_status st0 = check_args(Q, K, V, O, LSE, B, H, N, d, scale);
+  if (st0 != FA_OK) return st0;
+  if (workspace == nullptr) return FA_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 15u) != 0) return FA_ERR_ALIGN;
+  if (num_splits <= 0) num_splits = default_splits(B, H, N, causal != 0);
+  if (num_splits > kMaxSplits) return FA_ERR_UNSUPPORTED;
+  // equal ranges of key tiles; trailing empty ranges are dropped
+  const int n_kv = (N + kBN - 1) / kBN;
+  const int kv_per_split = (n_kv + num_splits - 1) / num_splits;
+  num_splits = (n_kv + kv_per_split - 1) / kv_per_split;
+  const size_t need = splitkv_bytes(B, H, N, d, num_splits);
+  if (workspace_bytes < need) return FA_ERR_WORKSPACE;
+  const size_t nbytes = static_cast<size_t>(B) * H * N * d * 2;
+  if (overlaps(workspace, need, Q, nbytes) || overlaps(workspace, need, K, nbytes) ||
+      overlaps(workspace, need, V, nbytes) || overlaps(workspace, need, O, nbytes) ||
+      (LSE && overlaps(workspace, need, LSE, static_cast<size_t>(B) * H * N * 4)))
+    return FA_ERR_ALIAS;
+  st0 = prepare(LSE, B, H, N, d, scale, &prm, &dev);
+  if (st0 != FA_OK) return st0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int bh = prm.BH;
+  if (num_splits == 1) {
+    // one range: the fused kernel writes O and LSE directly
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (d == 128)
+      return causal ? launch<128, true, false>(Q, K, V, O, prm, N, bh, st, *dev)
+                    : launch<128, false, false>(Q, K, V, O, prm, N, bh, st, *dev);
+    return causal ? launch<64, true, false>(Q, K, V, O, prm, N, bh, st, *dev)
+                  : launch<64, false, false>(Q, K, V, O, prm, N, bh, st, *dev);
+  }
+  const long long rows = splitkv_rows(B, H, N);
+  prm.num_splits = num_splits;
+  prm.kv_per_split = kv_per_split;
+  prm.o_part = static_cast<float*>(workspace);
+  prm.lse_part = prm.o_part + static_cast<size_t>(num_splits) * rows * d;
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  fa_status r;
+  if (d == 128)
+    r = causal ? launch<128, true, true>(Q, K, V, O, prm, N, bh, st, *dev)
+               : launch<128, false, true>(Q, K, V, O, prm, N, bh, st, *dev);
+  else
+    r = causal ? launch<64, true, true>(Q, K, V, O, prm, N, bh, st, *dev)
+               : launch<64, false, true>(Q, K, V, O, prm, N, bh, st, *dev);
+  if (r != FA_OK) return r;
+  return d == 128 ? launch_merge<128>(prm.o_part, prm.lse_part, O, LSE, rows, num_splits, st)
+                  : launch_merge<64>(prm.o_part, prm.lse_part, O, LSE, rows, num_splits, st);
 }
 
 fa_status fa_get_device_status_word(void* stream, unsigned int* word) {

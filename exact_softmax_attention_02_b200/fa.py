@@ -59,6 +59,13 @@ def _load():
     lib.fa_last_cuda_error.restype = ctypes.c_char_p
     lib.fa_set_debug.argtypes = [ctypes.c_uint, ctypes.c_ulonglong]
     lib.fa_set_debug.restype = None
+    lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_size_t, c_int, c_int, c_int,
+                                   c_int, c_float, c_int, c_int, vp]
+    lib.fa_fwd_splitkv.restype = c_int
+    lib.fa_fwd_splitkv_workspace_bytes.argtypes = [c_int, c_int, c_int, c_int, c_int, c_int]
+    lib.fa_fwd_splitkv_workspace_bytes.restype = ctypes.c_size_t
+    lib.fa_fwd_splitkv_default_splits.argtypes = [c_int, c_int, c_int, c_int, c_int]
+    lib.fa_fwd_splitkv_default_splits.restype = c_int
     lib.fa_version.argtypes = []
     lib.fa_version.restype = ctypes.c_char_p
     _lib = lib
@@ -116,9 +123,61 @@ def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
                       B, H, N, d, float(scale), int(bool(causal)), _stream_handle(stream)))
 
 
+def _check_qkvo(q, k, v, o):
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if t.dim() != 4:
+            raise ValueError(f"{name} must be [B, H, N, d]")
+    if not (q.shape == k.shape == v.shape == o.shape):
+        raise ValueError(f"shape mismatch: q{tuple(q.shape)} k{tuple(k.shape)} "
+                         f"v{tuple(v.shape)} o{tuple(o.shape)}")
+
+
+def splitkv_workspace_bytes(B: int, H: int, N: int, d: int, num_splits: int = 0,
+                            causal: bool = False) -> int:
+    """Workspace bytes fa_fwd_splitkv needs (num_splits <= 0: the default)."""
+    return int(_load().fa_fwd_splitkv_workspace_bytes(B, H, N, d, int(bool(causal)), num_splits))
+
+
+def splitkv_default_splits(B: int, H: int, N: int, d: int, causal: bool = False) -> int:
+    return int(_load().fa_fwd_splitkv_default_splits(B, H, N, d, int(bool(causal))))
+
+
+def fa_fwd_splitkv(q, k, v, o, lse=None, workspace=None, num_splits: int = 0,
+                   scale: float | None = None, causal: bool = False, stream=None) -> None:
+    """Split-KV forward (same result as fa_fwd).  ``workspace``: a CUDA tensor
+    of at least splitkv_workspace_bytes(...) bytes (allocated here if None)."""
+    lib = _load()
+    _check_qkvo(q, k, v, o)
+    B, H, N, d = q.shape
+    lse_ptr = None
+    if lse is not None:
+        if lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous():
+            raise ValueError("lse must be a contiguous CUDA float32 tensor")
+        if tuple(lse.shape) != (B, H, N):
+            raise ValueError(f"lse must be [B, H, N] = {(B, H, N)}")
+        lse_ptr = lse.data_ptr()
+    if workspace is None:
+        nbytes = splitkv_workspace_bytes(B, H, N, d, num_splits, causal)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    _check(lib.fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_ptr,
+                              workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                              B, H, N, d, float(scale), int(bool(causal)), int(num_splits),
+                              _stream_handle(stream)))
+
+
 def attention_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                       scale: float | None = None, causal: bool = False,
-                      return_lse: bool = True, device=None, out=None):
+                      return_lse: bool = True, device=None, out=None, num_splits=None):
     """Allocate the outputs and run the forward.
 
     CUDA inputs: outputs stay on their device.  CPU inputs (ideally pinned):
@@ -126,7 +185,8 @@ def attention_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     kernel runs there, and O (and LSE) are copied back to host memory -- into
     ``out = (o_host, lse_host)`` when given (pinned buffers of the right shape
     and dtype, reused across calls), else into new pinned tensors.  The call
-    returns after the copies have completed.
+    returns after the copies have completed.  ``num_splits`` (not None) runs
+    the split-KV forward with that many key ranges (0: its default).
     """
     on_host = not q.is_cuda
     if on_host:
@@ -137,7 +197,10 @@ def attention_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         v = v.to(dev, non_blocking=True)
     o = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if return_lse else None
-    fa_fwd(q, k, v, o, lse, scale=scale, causal=causal)
+    if num_splits is None:
+        fa_fwd(q, k, v, o, lse, scale=scale, causal=causal)
+    else:
+        fa_fwd_splitkv(q, k, v, o, lse, num_splits=num_splits, scale=scale, causal=causal)
     if not on_host:
         return (o, lse) if return_lse else o
     if out is not None:

@@ -59,6 +59,9 @@ WORKLOADS = {
         Workload("b1h32n32768d128_causal_q4", 1, 32, 32768, 128, True, 3, q_std=4.0,
                  sample_rows=2048),
         Workload("b1h8n131072d128_causal", 1, 8, 131072, 128, True, 4, sample_rows=1024),
+        # few query blocks for 148 SMs: the shapes the split-KV path is for
+        Workload("b1h2n8192d128", 1, 2, 8192, 128, False, 5, sample_rows=1024),
+        Workload("b1h1n32768d128_causal", 1, 1, 32768, 128, True, 6, sample_rows=1024),
     )
 }
 

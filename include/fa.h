@@ -27,6 +27,8 @@
 #ifndef FA_H_
 #define FA_H_
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -39,7 +41,8 @@ typedef enum fa_status {
   FA_ERR_ALIGN = 4,           /* a pointer is not 16-byte aligned (LSE: 4-byte)   */
   FA_ERR_CUDA = 5,            /* a CUDA runtime/driver call or the launch failed  */
   FA_ERR_DEVICE_TIMEOUT = 6,  /* a kernel gave up on a bounded wait               */
-  FA_ERR_ALIAS = 7            /* O or LSE overlaps an input or each other         */
+  FA_ERR_ALIAS = 7,           /* O, LSE or a workspace overlaps another argument  */
+  FA_ERR_WORKSPACE = 8        /* the workspace is smaller than required           */
 } fa_status;
 
 /*
@@ -68,6 +71,47 @@ typedef enum fa_status {
  */
 fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H,
                  int N, int d, float scale, int causal, void* stream);
+
+/*
+ * fa_fwd_splitkv -- the same result as fa_fwd, with the key range of every
+ * query block divided into num_splits ranges processed by separate CTAs, for
+ * problems with too few query blocks to fill the GPU.  Each range leaves a
+ * partial state -- its normalised output u/l and its log-sum-exp -- and a
+ * second kernel merges the states of a row: with M = max_s LSE_s and
+ * w_s = e^(LSE_s - M) (0 for a range with no allowed key), O = sum w_s O_s /
+ * sum w_s and LSE = M + ln sum w_s.  This is the block update of liminalml.com
+ * "FlashAttention" (rescale both numerator and denominator by e^(m - m')) and
+ * the block merge of interactiveml.org (old scale 0 while m = -inf), applied
+ * to whole partial states.
+ *
+ *   Q, K, V, O, LSE, B, H, N, d, scale, causal, stream: as for fa_fwd.
+ *   workspace        device memory owned by the caller, 16-byte aligned, at
+ *                    least fa_fwd_splitkv_workspace_bytes(B, H, N, d,
+ *                    causal, num_splits) bytes; overwritten (fp32 partial outputs
+ *                    [splits][B*H*N][d] followed by partial LSE
+ *                    [splits][B*H*N]); must not overlap any other argument.
+ *   workspace_bytes  its size.
+ *   num_splits       1..256; <= 0 picks fa_fwd_splitkv_default_splits().
+ *                    Ranges are ceil(ceil(N/128) / num_splits) key tiles;
+ *                    trailing empty ranges are dropped.  When one range
+ *                    remains, the fused kernel of fa_fwd runs and the
+ *                    workspace is not touched.
+ * Errors as fa_fwd, plus FA_ERR_NULL for a NULL workspace, FA_ERR_ALIGN for a
+ * misaligned one, FA_ERR_WORKSPACE when it is too small, FA_ERR_UNSUPPORTED
+ * for num_splits > 256.  Two kernels are enqueued on `stream`.
+ */
+fa_status fa_fwd_splitkv(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                         void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+                         float scale, int causal, int num_splits, void* stream);
+
+/* Bytes of workspace fa_fwd_splitkv needs (0 for invalid arguments).
+ * num_splits <= 0 means the default for this shape and mask. */
+size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int N, int d, int causal, int num_splits);
+
+/* Default split count: non-causal, the most ranges that fit in one wave of
+ * 148 SMs; causal, at least 1.5 waves; at least two key tiles per range
+ * (1 for invalid arguments). */
+int fa_fwd_splitkv_default_splits(int B, int H, int N, int d, int causal);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fa_status_string(fa_status status);

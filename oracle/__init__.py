@@ -12,6 +12,7 @@ from .attention import (  # noqa: F401
     brute_force_attention,
     flops_for_rows,
     merge_block,
+    merge_states,
     online_attention_rows,
     scalar_online_weighted_sum,
     scalar_softmax_weighted_sum,

@@ -42,6 +42,11 @@ Three functions, three independent computations:
 * ``brute_force_attention`` -- pure-Python loops, no max subtraction, exact
   summation with ``math.fsum``; only for tiny inputs.
 
+``attention_rows(..., key_range=(lo, hi))`` gives the partial state of one
+key range, and ``merge_states`` folds such states together (the block update
+applied to whole states); merged states over disjoint ranges equal the full
+row (pinned in tests/test_oracle_pins.py).
+
 Inputs are arrays of shape [B, H, N, d] of any real dtype (bf16 values
 widened to float32 or float64 are exact); they are converted to float64 here.
 
@@ -57,6 +62,7 @@ import numpy as np
 
 __all__ = [
     "attention_rows",
+    "merge_states",
     "attention_full",
     "online_attention_rows",
     "merge_block",
@@ -90,7 +96,7 @@ def _group_rows(rows: np.ndarray):
         yield b, h, pos, rows[pos, 2]
 
 
-def attention_rows(q, k, v, scale: float, causal: bool, rows):
+def attention_rows(q, k, v, scale: float, causal: bool, rows, key_range=None):
     """Exact attention output and LSE for the selected rows.
 
     Follows the dense definition O = softmax(scale * Q K^T) V
@@ -104,6 +110,9 @@ def attention_rows(q, k, v, scale: float, causal: bool, rows):
       scale:   multiplier of the dot product (1/sqrt(d) by default upstream).
       causal:  if true, query i sees keys j <= i only.
       rows:    int array [R, 3] of (b, h, i).
+      key_range: optional (lo, hi): only keys lo <= j < hi are allowed (the
+               partial state of one key range).  A row with no allowed key
+               gets O = 0 and LSE = -inf (the empty state, weight 0 in a merge).
 
     Returns:
       (O, LSE): float64 arrays [R, d] and [R].
@@ -122,14 +131,20 @@ def attention_rows(q, k, v, scale: float, causal: bool, rows):
             i = qi[c0:c0 + chunk]
             Q = _as_f64(q[b, h][i])  # [r, d]
             s = scale * (Q @ K.T)  # [r, N]   the score rows
+            j = np.arange(n_keys)
             if causal:
-                j = np.arange(n_keys)
                 s = np.where(j[None, :] <= i[:, None], s, -np.inf)
+            if key_range is not None:
+                lo, hi = key_range
+                s = np.where((j[None, :] >= lo) & (j[None, :] < hi), s, -np.inf)
             m = s.max(axis=1)  # largest score of each row
-            w = np.exp(s - m[:, None])  # weights relative to it; masked -> 0
+            empty = np.isneginf(m)
+            m_safe = np.where(empty, 0.0, m)
+            w = np.exp(s - m_safe[:, None])  # weights relative to it; masked -> 0
             z = w.sum(axis=1)  # denominator
-            out[p] = (w @ V) / z[:, None]
-            lse[p] = m + np.log(z)
+            with np.errstate(invalid="ignore", divide="ignore"):
+                out[p] = np.where(empty[:, None], 0.0, (w @ V) / z[:, None])
+                lse[p] = np.where(empty, -np.inf, m + np.log(z))
     return out, lse
 
 
@@ -170,6 +185,36 @@ def merge_block(m, total, acc, scores, values):
     total = total * old_scale + weight.sum(axis=1)
     acc = acc * old_scale[:, None] + weight @ values
     return new_max, total, acc
+
+
+def merge_states(o_parts, lse_parts):
+    """Merge partial attention states of the same rows over disjoint key ranges.
+
+    Each state s is a normalised partial output O_s = u_s / l_s and its
+    log-sum-exp LSE_s = m_s + ln l_s.  Folding them in one after another is
+    the block update with whole states as blocks (liminalml.com
+    "FlashAttention": m' = max(m, m_s), both the running numerator and
+    denominator rescaled by e^(m - m'); interactiveml.org: the old scale is 0
+    while m = -inf).  An empty state (LSE = -inf) has weight 0.
+
+    Args: o_parts [S, R, d], lse_parts [S, R].  Returns (O [R, d], LSE [R]).
+    """
+    o_parts = np.asarray(o_parts, dtype=np.float64)
+    lse_parts = np.asarray(lse_parts, dtype=np.float64)
+    m = np.full(lse_parts.shape[1], -np.inf)
+    total = np.zeros(lse_parts.shape[1])
+    acc = np.zeros(o_parts.shape[1:])
+    with np.errstate(invalid="ignore"):
+        for o_s, l_s in zip(o_parts, lse_parts):
+            new_m = np.maximum(m, l_s)
+            old_scale = np.where(np.isneginf(m), 0.0, np.exp(m - new_m))
+            weight = np.where(np.isneginf(l_s), 0.0, np.exp(l_s - np.where(np.isneginf(new_m), 0.0, new_m)))
+            total = total * old_scale + weight
+            acc = acc * old_scale[:, None] + weight[:, None] * o_s
+            m = new_m
+        out = np.where(total[:, None] > 0, acc / np.where(total > 0, total, 1.0)[:, None], 0.0)
+        lse = np.where(total > 0, m + np.log(np.where(total > 0, total, 1.0)), -np.inf)
+    return out, lse
 
 
 def online_attention_rows(q, k, v, scale: float, causal: bool, rows, tile: int = 64):

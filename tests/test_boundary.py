@@ -16,7 +16,7 @@ HEADER = os.path.join(ROOT, "include", "fa.h")
 LIB = os.path.join(ROOT, "exact_softmax_attention_02_b200", "libfa.so")
 
 FA_OK, FA_ERR_NULL, FA_ERR_SHAPE, FA_ERR_UNSUPPORTED, FA_ERR_ALIGN = 0, 1, 2, 3, 4
-FA_ERR_CUDA, FA_ERR_DEVICE_TIMEOUT, FA_ERR_ALIAS = 5, 6, 7
+FA_ERR_CUDA, FA_ERR_DEVICE_TIMEOUT, FA_ERR_ALIAS, FA_ERR_WORKSPACE = 5, 6, 7, 8
 
 
 @pytest.fixture(scope="module")
@@ -53,7 +53,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(8):
+    for code in range(9):
         s = lib.fa_status_string(code).decode()
         assert s.startswith("FA_")
     assert lib.fa_status_string(99).decode() == "unknown fa_status"
@@ -108,3 +108,46 @@ def test_aliasing(lib):
     assert call(lib, lse=A + 192 * MB + 1024) == FA_ERR_ALIAS
     # LSE overlapping V
     assert call(lib, lse=A + 128 * MB) == FA_ERR_ALIAS
+
+
+# split-KV entry point: workspace checks run before any device call
+def _splitkv(lib, ws=A + 512 * MB, ws_bytes=1 << 30, num_splits=2, **kw):
+    lib.fa_fwd_splitkv.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_size_t] + [ctypes.c_int] * 4 + \
+        [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+    lib.fa_fwd_splitkv.restype = ctypes.c_int
+    args = dict(q=A, k=A + 64 * MB, v=A + 128 * MB, o=A + 192 * MB, lse=A + 256 * MB,
+                B=1, H=1, N=1024, d=64, scale=0.125, causal=0)
+    args.update(kw)
+    return lib.fa_fwd_splitkv(args["q"], args["k"], args["v"], args["o"], args["lse"], ws, ws_bytes,
+                              args["B"], args["H"], args["N"], args["d"], args["scale"],
+                              args["causal"], num_splits, None)
+
+
+def test_splitkv_workspace_checks(lib):
+    lib.fa_fwd_splitkv_workspace_bytes.argtypes = [ctypes.c_int] * 6
+    lib.fa_fwd_splitkv_workspace_bytes.restype = ctypes.c_size_t
+    need = lib.fa_fwd_splitkv_workspace_bytes(1, 1, 1024, 64, 0, 2)
+    assert need == 2 * 1024 * (64 + 1) * 4
+    assert lib.fa_fwd_splitkv_workspace_bytes(1, 1, 1024, 96, 0, 2) == 0
+    # the default split count depends on the mask
+    assert lib.fa_fwd_splitkv_workspace_bytes(1, 2, 8192, 128, 1, 0) == 4 * 2 * 8192 * 129 * 4
+    assert _splitkv(lib, ws=None) == FA_ERR_NULL
+    assert _splitkv(lib, ws=A + 512 * MB + 4) == FA_ERR_ALIGN
+    assert _splitkv(lib, ws_bytes=need - 4) == FA_ERR_WORKSPACE
+    assert _splitkv(lib, num_splits=300) == FA_ERR_UNSUPPORTED
+    assert _splitkv(lib, ws=A + 128 * MB + 1024) == FA_ERR_ALIAS  # inside V
+    assert _splitkv(lib, q=None) == FA_ERR_NULL
+    assert _splitkv(lib, d=32) == FA_ERR_UNSUPPORTED
+
+
+def test_splitkv_default_splits(lib):
+    lib.fa_fwd_splitkv_default_splits.argtypes = [ctypes.c_int] * 5
+    lib.fa_fwd_splitkv_default_splits.restype = ctypes.c_int
+    # 2 heads x 32 query blocks = 64 CTAs: one wave of 148 SMs (1.5 causal)
+    assert lib.fa_fwd_splitkv_default_splits(1, 2, 8192, 128, 0) == 2
+    assert lib.fa_fwd_splitkv_default_splits(1, 2, 8192, 128, 1) == 4
+    assert lib.fa_fwd_splitkv_default_splits(1, 1, 32768, 128, 1) == 2
+    # already many CTAs: no split
+    assert lib.fa_fwd_splitkv_default_splits(4, 16, 4096, 64, 0) == 1
+    # at least two key tiles per range
+    assert lib.fa_fwd_splitkv_default_splits(1, 1, 512, 64, 0) == 2

@@ -386,3 +386,56 @@ def test_pins_reject_merge_without_rescale():
     finally:
         A.merge_block = real
     assert fails
+
+
+# ---------------------------------------------------------------------------
+# Partial states over key ranges, and their merge
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_merge_of_key_range_states_is_full_attention(causal):
+    """Attention over disjoint key ranges, merged, equals attention over all keys."""
+    from oracle import merge_states
+
+    rng = np.random.default_rng(11)
+    B, H, N, d = 1, 2, 300, 8
+    q = rng.standard_normal((B, H, N, d)) * 2
+    k = rng.standard_normal((B, H, N, d))
+    v = rng.standard_normal((B, H, N, d))
+    rows = all_rows(B, H, N)
+    full_o, full_l = attention_rows(q, k, v, 0.4, causal, rows)
+    bounds = [0, 1, 128, 129, 256, 300]
+    parts = [attention_rows(q, k, v, 0.4, causal, rows, key_range=(lo, hi))
+             for lo, hi in zip(bounds[:-1], bounds[1:])]
+    o, l = merge_states([p[0] for p in parts], [p[1] for p in parts])
+    assert np.allclose(o, full_o, rtol=1e-12, atol=1e-13)
+    assert np.allclose(l, full_l, rtol=1e-12, atol=1e-13)
+    # the order of the states does not matter
+    o2, l2 = merge_states([p[0] for p in parts[::-1]], [p[1] for p in parts[::-1]])
+    assert np.allclose(o2, full_o, rtol=1e-12, atol=1e-13)
+    if causal:
+        # rows before a range's first key have an empty state there
+        assert np.isneginf(parts[-1][1][:256]).all() and (parts[-1][0][:256] == 0).all()
+
+
+def test_key_range_state_closed_form():
+    """One key in range: the state is that key's value and its score."""
+    q, k, v = scalar_problem([0.0, 1.0, 2.0], [10.0, 20.0, 30.0])
+    o, l = attention_rows(q, k, v, 1.0, False, all_rows(1, 1, 3), key_range=(1, 2))
+    assert (o[:, 0] == 20.0).all() and (l == 1.0).all()
+    o, l = attention_rows(q, k, v, 1.0, False, all_rows(1, 1, 3), key_range=(3, 3))
+    assert (o == 0).all() and np.isneginf(l).all()
+
+
+def test_merge_rejects_missing_rescale():
+    """A merge that does not rescale the old accumulator is caught by the pin."""
+    from oracle import merge_states
+
+    q, k, v = scalar_problem([0.0, 1.0, 2.0], [10.0, 20.0, 30.0])
+    rows = all_rows(1, 1, 3)
+    parts = [attention_rows(q, k, v, 1.0, False, rows, key_range=(lo, lo + 1)) for lo in range(3)]
+    o, _ = merge_states([p[0] for p in parts], [p[1] for p in parts])
+    assert round(o[0, 0], 6) == 25.752104
+    # planted mistake: plain average of the partial outputs (block averaging)
+    bad = np.mean([p[0] for p in parts], axis=0)
+    assert abs(bad[0, 0] - o[0, 0]) > 1.0
