@@ -1039,6 +1039,69 @@ fa_status fa_fwd_splitkv(const void* Q, const void* K, const void* V, void* O, f
                   : launch_merge<64>(prm.o_part, prm.lse_part, O, LSE, rows, num_splits, st);
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// split-KV without any allocation
+// ---------------------------------------------------------------------------
+// Some callers cannot allocate device memory at the moment they need
+// attention: code running inside a CUDA stream capture that must not add
+// allocation nodes, real-time or embedded runtimes that forbid allocation
+// after start-up, or hosts whose memory pool is owned by another framework.
+// For them the split-KV forward can run on a workspace that is part of this
+// library: a fixed array in device memory, allocated once when the library's
+// code is loaded on a GPU and held by every GPU that loads it until the
+// process exits.
+namespace fa {
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on each device.  In host code the
+// array's name is only a stand-in for the symbol, never an address a kernel
+// may use; the real address is looked up once per device, with that device
+// current.
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+}  // namespace
+}  // namespace fa
+
+extern "C" {
+
+fa_status fa_fwd_splitkv_noalloc(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                                 int B, int H, int N, int d, float scale, int causal, int num_splits,
+                                 void* stream) {
+  using namespace fa;
+  // argument errors are reported exactly as fa_fwd_splitkv reports them
+  fa_status st0 = check_args(Q, K, V, O, LSE, B, H, N, d, scale);
+  if (st0 != FA_OK) return st0;
+  if (num_splits > kMaxSplits) return FA_ERR_UNSUPPORTED;
+  const size_t need = fa_fwd_splitkv_workspace_bytes(B, H, N, d, causal, num_splits);
+  if (need > static_cast<size_t>(FA_NOALLOC_SCRATCH_BYTES)) return FA_ERR_WORKSPACE;
+  int dev_id = 0;
+  cudaError_t e = cudaGetDevice(&dev_id);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev_id < 0 || dev_id >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev_id] == nullptr) {
+      // first call on this device: find the array's device address
+      e = cudaGetSymbolAddress(&g_noalloc_ptr[dev_id], g_noalloc_scratch);
+      if (e != cudaSuccess) {
+        g_noalloc_ptr[dev_id] = nullptr;
+        return cuda_fail(e, "cudaGetSymbolAddress");
+      }
+    }
+    scratch = g_noalloc_ptr[dev_id];
+  }
+  // Every partial state the merge reads is written first by the same call,
+  // so nothing in the scratch has to start at zero.
+  return fa_fwd_splitkv(Q, K, V, O, LSE, scratch, static_cast<size_t>(FA_NOALLOC_SCRATCH_BYTES), B,
+                        H, N, d, scale, causal, num_splits, stream);
+}
+
 fa_status fa_get_device_status_word(void* stream, unsigned int* word) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (word) *word = 0;

@@ -113,6 +113,40 @@ size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int N, int d, int causal, in
  * (1 for invalid arguments). */
 int fa_fwd_splitkv_default_splits(int B, int H, int N, int d, int causal);
 
+/* Size of the workspace built into the library for fa_fwd_splitkv_noalloc. */
+#define FA_NOALLOC_SCRATCH_BYTES (64 * 1024 * 1024)
+
+/*
+ * fa_fwd_splitkv_noalloc -- fa_fwd_splitkv for callers that cannot allocate
+ * device memory when they run attention: code being captured into a CUDA
+ * graph that must not gain allocation nodes, runtimes that forbid allocation
+ * after start-up, or programs whose device memory belongs to another
+ * framework's pool.  The pages describe no such entry point; it has no
+ * counterpart there.
+ *
+ * Instead of a caller's workspace it uses an array of
+ * FA_NOALLOC_SCRATCH_BYTES (64 MiB) that is part of this library's device
+ * code: every GPU that loads the library holds that memory until the process
+ * exits.  The caller still passes Q, K, V, O and LSE, with the meaning,
+ * layout and errors of fa_fwd_splitkv (num_splits <= 0 picks the default).
+ *
+ *   - A problem whose workspace (fa_fwd_splitkv_workspace_bytes) exceeds
+ *     FA_NOALLOC_SCRATCH_BYTES is rejected with FA_ERR_WORKSPACE before
+ *     anything is enqueued.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and keeps it; make
+ *     that first call before any stream capture.  The library allocates
+ *     nothing, on any call.
+ *   - All calls on a device share the one array, which keeps whatever the
+ *     last call left in it (nothing in it needs to start at zero).  Calls
+ *     that may overlap on the GPU -- on different streams without ordering,
+ *     or from several host threads -- race on it and must be serialised by
+ *     the caller.
+ */
+fa_status fa_fwd_splitkv_noalloc(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                                 int B, int H, int N, int d, float scale, int causal, int num_splits,
+                                 void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fa_status_string(fa_status status);
 
