@@ -178,6 +178,15 @@ def tensor_peak():
         return FALLBACK_PEAK_TFLOPS, "fallback (1.59 PFLOP/s, earlier measurement on this pool)"
 
 
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:
+        return 6650.0, "fallback (6.65 TB/s, earlier measurement on this pool)"
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
@@ -327,6 +336,14 @@ def run_ours(args, w):
 
     splits = None
     launches_per_step = 1
+    std_events = None
+    if args.path == "standard":
+        from exact_softmax_attention_02_b200 import comparator
+
+        g = min(w.B * w.H, comparator.heads_per_group(w.N))
+        std_buffers = (torch.empty((g, w.N, w.N), dtype=torch.float32, device=dev),
+                       torch.empty((g, w.N, w.N), dtype=torch.bfloat16, device=dev))
+        launches_per_step = (w.B * w.H + g - 1) // g  # our softmax; the two GEMMs are cuBLAS'
     if args.path == "splitkv":
         splits = args.splits if args.splits > 0 else fa.splitkv_default_splits(w.B, w.H, w.N, w.d, w.causal)
         ws = torch.empty(max(16, fa.splitkv_workspace_bytes(w.B, w.H, w.N, w.d, splits, w.causal)),
@@ -334,7 +351,10 @@ def run_ours(args, w):
         launches_per_step = 1 if splits == 1 else 2  # split kernel + merge
 
     def step():
-        if splits is None:
+        if args.path == "standard":
+            comparator.standard_attention(q, k, v, o, lse, scale=w.scale, causal=w.causal,
+                                          buffers=std_buffers, softmax_events=std_events)
+        elif splits is None:
             fa.fa_fwd(q, k, v, o, lse, scale=w.scale, causal=w.causal, stream=stream)
         else:
             fa.fa_fwd_splitkv(q, k, v, o, lse, workspace=ws, num_splits=splits, scale=w.scale,
@@ -353,6 +373,8 @@ def run_ours(args, w):
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize(dev)
+    if args.path == "standard":
+        std_events = []
     t_start.record(stream)
     for i in range(args.steps):
         ev[i][0].record(stream)
@@ -375,17 +397,27 @@ def run_ours(args, w):
     lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
     q_p, k_p, v_p = (t.pin_memory() for t in (q_h, k_h, v_h))
     e2e_steps = max(3, min(args.steps, 20))
+    def api_call():
+        if args.path == "standard":
+            qd, kd, vd = (t.to(dev, non_blocking=True) for t in (q_p, k_p, v_p))
+            od, ld = comparator.standard_attention(qd, kd, vd, scale=w.scale, causal=w.causal,
+                                                   buffers=std_buffers)
+            o_h.copy_(od, non_blocking=True)
+            lse_h.copy_(ld, non_blocking=True)
+            torch.cuda.current_stream(dev).synchronize()
+        else:
+            fa.attention_forward(q_p, k_p, v_p, scale=w.scale, causal=w.causal, out=(o_h, lse_h),
+                                 num_splits=splits)
+
     for _ in range(2):
-        fa.attention_forward(q_p, k_p, v_p, scale=w.scale, causal=w.causal, out=(o_h, lse_h),
-                             num_splits=splits)
+        api_call()
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        fa.attention_forward(q_p, k_p, v_p, scale=w.scale, causal=w.causal, out=(o_h, lse_h),
-                             num_splits=splits)
+        api_call()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist, dev)
@@ -397,6 +429,22 @@ def run_ours(args, w):
     peak, peak_src = tensor_peak()
     achieved = w.flops / avg_launch_s / 1e12
     traffic = committed_traffic(w.name)
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
+                "kernel": f"fa_fwd_kernel<{w.d},{str(w.causal).lower()}>"
+                          + (" + fa_merge_kernel" if args.path == "splitkv" and launches_per_step == 2 else ""),
+                "kernel_source_sha256": kernel_source_hash()}
+    if args.path == "standard":
+        # the comparator's dominant kernel is the HBM-bound row softmax:
+        # it reads the fp32 scores and writes the bf16 probabilities and LSE
+        sm_ms = [a.elapsed_time(b) for a, b in std_events]
+        sm_s = max_over_ranks(sum(sm_ms) / 1e3 / args.steps, dist, dev)
+        nbytes = w.B * w.H * w.N * (6 * w.N + 4)
+        hbm, hbm_src = hbm_peak()
+        roofline = {"bound": "hbm", "achieved": nbytes / sm_s / 1e9, "peak": hbm, "unit": "GB/s",
+                    "frac": nbytes / sm_s / 1e9 / hbm, "traffic": None, "peak_source": hbm_src,
+                    "kernel": "fa_std::softmax_rows_kernel", "algorithmic_bytes": nbytes,
+                    "step_tflops": achieved}
     launches = int(sum_over_ranks(args.steps * launches_per_step, dist, dev))
 
     cpu = None
@@ -418,11 +466,7 @@ def run_ours(args, w):
                        "l2": (f"inputs+outputs {in_bytes / 1e6:.0f} MB > L2 126 MB, no flush"
                               if in_bytes > L2_BYTES else "L2 not flushed (inputs < L2)")},
             "pct_of_peak": 100.0 * value / world / peak,
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
-                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": peak_src,
-                         "kernel": f"fa_fwd_kernel<{w.d},{str(w.causal).lower()}>" + (" + fa_merge_kernel" if launches_per_step == 2 else ""),
-                         "kernel_source_sha256": kernel_source_hash()},
+            "roofline": roofline,
             "e2e": {"value": weak_scaling_value(w.flops, world, e2e_steps, e2e_s), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
@@ -445,8 +489,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--path", default="fused", choices=["fused", "splitkv"],
-                    help="fused: fa_fwd; splitkv: fa_fwd_splitkv (key ranges + merge)")
+    ap.add_argument("--path", default="fused", choices=["fused", "splitkv", "standard"],
+                    help="fused: fa_fwd; splitkv: fa_fwd_splitkv (key ranges + merge); "
+                         "standard: the materialising comparator (GEMM, softmax, GEMM)")
     ap.add_argument("--splits", type=int, default=0, help="splitkv: key ranges (0 = default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-step-seconds", type=float, default=8.0,

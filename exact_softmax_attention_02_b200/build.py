@@ -2,8 +2,9 @@
 
     python -m exact_softmax_attention_02_b200.build [--force] [--verbose]
 
-The library is a single translation unit (csrc/fa_fwd.cu) linked against the
-static CUDA runtime; the driver entry point for tensor-map encoding is looked
+The library is built from csrc/fa_fwd.cu (the fused forward, split-KV and
+merge) and csrc/standard_softmax.cu (the comparator's softmax), linked
+against the static CUDA runtime; the driver entry point for tensor-map encoding is looked
 up at run time, so no libcuda link is needed.
 """
 
@@ -17,7 +18,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = [os.path.join(HERE, "csrc", "fa_fwd.cu")]
+SOURCES = [os.path.join(HERE, "csrc", "fa_fwd.cu"), os.path.join(HERE, "csrc", "standard_softmax.cu")]
 DEPENDS = SOURCES + [os.path.join(HERE, "csrc", "sm100.cuh"), os.path.join(ROOT, "include", "fa.h")]
 OUTPUT = os.path.join(HERE, "libfa.so")
 

@@ -62,6 +62,8 @@ WORKLOADS = {
         # few query blocks for 148 SMs: the shapes the split-KV path is for
         Workload("b1h2n8192d128", 1, 2, 8192, 128, False, 5, sample_rows=1024),
         Workload("b1h1n32768d128_causal", 1, 1, 32768, 128, True, 6, sample_rows=1024),
+        # small enough for multi-pass ncu captures of the materialising comparator
+        Workload("b1h4n4096d128_causal", 1, 4, 4096, 128, True, 7, sample_rows=1024),
     )
 }
 

@@ -147,6 +147,25 @@ fa_status fa_fwd_splitkv_noalloc(const void* Q, const void* K, const void* V, vo
                                  int B, int H, int N, int d, float scale, int causal, int num_splits,
                                  void* stream);
 
+/*
+ * fa_softmax_rows -- the softmax step of standard (materialising) attention,
+ * kept as a comparator: standard attention writes the N x N scores to
+ * global memory, reads them back for the softmax, writes the probabilities
+ * and reads them again for the product with V (sadullah.online "Flash
+ * Attention Explained", the memory-movement section; interactiveml.org, the
+ * square table of scores written to and read back from HBM).
+ *
+ *   S    device, fp32 [BH][N][N], read: the raw dot products q_i . k_j.
+ *   P    device, bf16 [BH][N][N], written: softmax_j(scale * S[i][j]) over the
+ *        allowed keys (j <= i when causal), 0 elsewhere.
+ *   LSE  device, fp32 [BH][N], written (may be NULL): ln sum_j e^(scale S_ij).
+ *   N    must be even (rows of P stay 4-byte aligned); scale > 0.
+ * Asynchronous on `stream`.  FA_ERR_NULL / _SHAPE / _UNSUPPORTED / _ALIGN
+ * for bad arguments, FA_ERR_CUDA if the launch fails.
+ */
+fa_status fa_softmax_rows(const float* S, void* P, float* LSE, int BH, int N, float scale,
+                          int causal, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fa_status_string(fa_status status);
 
