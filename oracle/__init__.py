@@ -7,6 +7,7 @@ the product.
 """
 
 from .attention import (  # noqa: F401
+    attention_backward,
     attention_full,
     attention_rows,
     brute_force_attention,

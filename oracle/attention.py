@@ -42,6 +42,9 @@ Three functions, three independent computations:
 * ``brute_force_attention`` -- pure-Python loops, no max subtraction, exact
   summation with ``math.fsum``; only for tiny inputs.
 
+``attention_backward`` gives dQ, dK, dV of L = sum(O * dO), the derivative
+of the same definition (pinned by finite differences).
+
 ``attention_rows(..., key_range=(lo, hi))`` gives the partial state of one
 key range, and ``merge_states`` folds such states together (the block update
 applied to whole states); merged states over disjoint ranges equal the full
@@ -62,6 +65,7 @@ import numpy as np
 
 __all__ = [
     "attention_rows",
+    "attention_backward",
     "merge_states",
     "attention_full",
     "online_attention_rows",
@@ -185,6 +189,50 @@ def merge_block(m, total, acc, scores, values):
     total = total * old_scale + weight.sum(axis=1)
     acc = acc * old_scale[:, None] + weight @ values
     return new_max, total, acc
+
+
+def attention_backward(q, k, v, do, scale: float, causal: bool):
+    """Gradients of L = sum(O * dO) with O = softmax(scale Q K^T [mask]) V.
+
+    The pages name the backward pass only ("selected recomputation in the
+    backward pass", lihaoran.work; "tiling, fusion, and recomputation",
+    liminalml.com "Why use it?").  What it computes is the derivative of the
+    forward definition, written out per head with the full score matrix:
+
+        P  = softmax(scale * Q K^T) over the allowed keys
+        dV = P^T dO
+        dP = dO V^T
+        D  = rowsum(dO * O)          (= rowsum(P * dP))
+        dS = P * (dP - D)
+        dQ = scale * dS K
+        dK = scale * dS^T Q
+
+    Args: q, k, v, do arrays [B, H, N, d].  Returns float64 (dQ, dK, dV, D),
+    D of shape [B, H, N].
+    """
+    B, H, N, d = np.shape(q)
+    dq = np.zeros((B, H, N, d))
+    dk = np.zeros((B, H, N, d))
+    dv = np.zeros((B, H, N, d))
+    dd = np.zeros((B, H, N))
+    for b in range(B):
+        for h in range(H):
+            Q, K, V, dO = (_as_f64(t[b, h]) for t in (q, k, v, do))
+            S = scale * (Q @ K.T)
+            if causal:
+                S = np.where(np.tril(np.ones((N, N), dtype=bool)), S, -np.inf)
+            M = S.max(axis=1, keepdims=True)
+            W = np.exp(S - M)
+            P = W / W.sum(axis=1, keepdims=True)
+            O = P @ V
+            dv[b, h] = P.T @ dO
+            dP = dO @ V.T
+            D = (dO * O).sum(axis=1)
+            dS = P * (dP - D[:, None])
+            dq[b, h] = scale * (dS @ K)
+            dk[b, h] = scale * (dS.T @ Q)
+            dd[b, h] = D
+    return dq, dk, dv, dd
 
 
 def merge_states(o_parts, lse_parts):

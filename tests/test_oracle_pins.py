@@ -439,3 +439,83 @@ def test_merge_rejects_missing_rescale():
     # planted mistake: plain average of the partial outputs (block averaging)
     bad = np.mean([p[0] for p in parts], axis=0)
     assert abs(bad[0, 0] - o[0, 0]) > 1.0
+
+
+# ---------------------------------------------------------------------------
+# Backward: gradients of L = sum(O * dO)
+# ---------------------------------------------------------------------------
+
+def _loss(q, k, v, do, scale, causal):
+    o, _ = attention_full(q, k, v, scale, causal)
+    return float((o * do).sum())
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_matches_finite_differences(causal):
+    from oracle import attention_backward
+
+    rng = np.random.default_rng(31 + int(causal))
+    B, H, N, d = 1, 2, 6, 3
+    q, k, v, do = (rng.standard_normal((B, H, N, d)) for _ in range(4))
+    scale = 0.8
+    dq, dk, dv, _ = attention_backward(q, k, v, do, scale, causal)
+    eps = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args = {"q": q, "k": k, "v": v}
+            args[name] = xp
+            lp = _loss(args["q"], args["k"], args["v"], do, scale, causal)
+            args[name] = xm
+            lm = _loss(args["q"], args["k"], args["v"], do, scale, causal)
+            num[idx] = (lp - lm) / (2 * eps)
+        assert np.allclose(g, num, rtol=1e-6, atol=1e-8), name
+
+
+def test_backward_closed_forms():
+    from oracle import attention_backward
+
+    rng = np.random.default_rng(8)
+    B, H, N, d = 1, 1, 7, 4
+    q = rng.standard_normal((B, H, N, d))
+    k = np.broadcast_to(rng.standard_normal((1, 1, 1, d)), (B, H, N, d)).copy()
+    v = rng.standard_normal((B, H, N, d))
+    do = rng.standard_normal((B, H, N, d))
+    for causal in (False, True):
+        dq, dk, dv, D = attention_backward(q, k, v, do, 0.6, causal)
+        # all keys equal: every score row is constant, so dQ = 0 exactly
+        assert np.allclose(dq, 0.0, atol=1e-13)
+        # uniform weights: dV_j = sum over queries that see j of dO_i / (#keys they see)
+        n_allowed = np.arange(1, N + 1) if causal else np.full(N, N)
+        for j in range(N):
+            rows = [i for i in range(N) if (not causal or j <= i)]
+            expect = sum(do[0, 0, i] / n_allowed[i] for i in rows)
+            assert np.allclose(dv[0, 0, j], expect, atol=1e-13)
+    # D = rowsum(dO * O) equals rowsum(P * dP): check against the forward
+    o, _ = attention_full(q, k, v, 0.6, False)
+    _, _, _, D = attention_backward(q, k, v, do, 0.6, False)
+    assert np.allclose(D, (o * do).sum(-1), rtol=1e-13)
+
+
+def test_backward_pins_reject_a_dropped_term():
+    """Leaving D out of dS is caught by the finite-difference pin."""
+    from oracle import attention_backward
+
+    rng = np.random.default_rng(2)
+    q, k, v, do = (rng.standard_normal((1, 1, 5, 3)) for _ in range(4))
+    dq, dk, dv, D = attention_backward(q, k, v, do, 1.0, False)
+    # rebuild dQ without the D term
+    S = q[0, 0] @ k[0, 0].T
+    P = np.exp(S - S.max(1, keepdims=True))
+    P /= P.sum(1, keepdims=True)
+    bad_dq = (P * (do[0, 0] @ v[0, 0].T)) @ k[0, 0]
+    eps = 1e-6
+    qp, qm = q.copy(), q.copy()
+    qp[0, 0, 2, 1] += eps
+    qm[0, 0, 2, 1] -= eps
+    num = (_loss(qp, k, v, do, 1.0, False) - _loss(qm, k, v, do, 1.0, False)) / (2 * eps)
+    assert abs(dq[0, 0, 2, 1] - num) < 1e-7
+    assert abs(bad_dq[2, 1] - num) > 1e-3
