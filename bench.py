@@ -344,6 +344,15 @@ def run_ours(args, w):
         std_buffers = (torch.empty((g, w.N, w.N), dtype=torch.float32, device=dev),
                        torch.empty((g, w.N, w.N), dtype=torch.bfloat16, device=dev))
         launches_per_step = (w.B * w.H + g - 1) // g  # our softmax; the two GEMMs are cuBLAS'
+    bwd = None
+    if args.path == "backward":
+        # one forward for O and LSE, then every step is one fa_bwd
+        fa.fa_fwd(q, k, v, o, lse, scale=w.scale, causal=w.causal, stream=stream)
+        g = torch.Generator(device="cpu").manual_seed(w.seed + 100)
+        do = torch.randn(q.shape, generator=g).to(torch.bfloat16).to(dev)
+        bwd = dict(do=do, dq=torch.empty_like(q), dk=torch.empty_like(q), dv=torch.empty_like(q),
+                   ws=torch.empty(max(16, w.B * w.H * w.N * 4), dtype=torch.uint8, device=dev))
+        launches_per_step = 3  # D = rowsum(dO*O), dK/dV, dQ
     if args.path == "splitkv":
         splits = args.splits if args.splits > 0 else fa.splitkv_default_splits(w.B, w.H, w.N, w.d, w.causal)
         ws = torch.empty(max(16, fa.splitkv_workspace_bytes(w.B, w.H, w.N, w.d, splits, w.causal)),
@@ -351,7 +360,10 @@ def run_ours(args, w):
         launches_per_step = 1 if splits == 1 else 2  # split kernel + merge
 
     def step():
-        if args.path == "standard":
+        if bwd is not None:
+            fa.fa_bwd(q, k, v, o, bwd["do"], lse, bwd["dq"], bwd["dk"], bwd["dv"], workspace=bwd["ws"],
+                      scale=w.scale, causal=w.causal, stream=stream)
+        elif args.path == "standard":
             comparator.standard_attention(q, k, v, o, lse, scale=w.scale, causal=w.causal,
                                           buffers=std_buffers, softmax_events=std_events)
         elif splits is None:
@@ -396,9 +408,23 @@ def run_ours(args, w):
     o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
     lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
     q_p, k_p, v_p = (t.pin_memory() for t in (q_h, k_h, v_h))
+    if bwd is not None:
+        o_hb = o.cpu().pin_memory()
+        do_hb = bwd["do"].cpu().pin_memory()
+        lse_hb = lse.cpu().pin_memory()
+        grads_h = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(3)]
     e2e_steps = max(3, min(args.steps, 20))
     def api_call():
-        if args.path == "standard":
+        if bwd is not None:
+            # end to end: host q, k, v, o, do, lse in; dq, dk, dv back to the host
+            dev_t = [t.to(dev, non_blocking=True) for t in (q_p, k_p, v_p, o_hb, do_hb)]
+            l_d = lse_hb.to(dev, non_blocking=True)
+            g_d = [torch.empty_like(dev_t[0]) for _ in range(3)]
+            fa.fa_bwd(*dev_t[:4], dev_t[4], l_d, *g_d, scale=w.scale, causal=w.causal)
+            for hbuf, dbuf in zip(grads_h, g_d):
+                hbuf.copy_(dbuf, non_blocking=True)
+            torch.cuda.current_stream(dev).synchronize()
+        elif args.path == "standard":
             qd, kd, vd = (t.to(dev, non_blocking=True) for t in (q_p, k_p, v_p))
             od, ld = comparator.standard_attention(qd, kd, vd, scale=w.scale, causal=w.causal,
                                                    buffers=std_buffers)
@@ -423,17 +449,26 @@ def run_ours(args, w):
     e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist, dev)
     h2d = 3 * q.numel() * q.element_size()
     d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+    if bwd is not None:
+        h2d = 5 * q.numel() * q.element_size() + lse.numel() * lse.element_size()
+        d2h = 3 * q.numel() * q.element_size()
 
     clocks = sampler.summary()
-    value = weak_scaling_value(w.flops, world, args.steps, elapsed_max)
+    # backward: five N^2 d products (2.5x the forward's two), the usual count
+    flops = w.flops * (2.5 if bwd is not None else 1.0)
+    value = weak_scaling_value(flops, world, args.steps, elapsed_max)
     peak, peak_src = tensor_peak()
-    achieved = w.flops / avg_launch_s / 1e12
+    achieved = flops / avg_launch_s / 1e12
     traffic = committed_traffic(w.name)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
                 "kernel": f"fa_fwd_kernel<{w.d},{str(w.causal).lower()}>"
                           + (" + fa_merge_kernel" if args.path == "splitkv" and launches_per_step == 2 else ""),
                 "kernel_source_sha256": kernel_source_hash()}
+    if bwd is not None:
+        # one step = rowdot + dK/dV + dQ kernels, timed together
+        roofline.update(kernel="bwd_rowdot + bwd_dkdv_kernel + bwd_dq_kernel", traffic=None,
+                        flops_convention="2.5 x forward (five N^2 d products)")
     if args.path == "standard":
         # the comparator's dominant kernel is the HBM-bound row softmax:
         # it reads the fp32 scores and writes the bf16 probabilities and LSE
@@ -448,7 +483,7 @@ def run_ours(args, w):
     launches = int(sum_over_ranks(args.steps * launches_per_step, dist, dev))
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and bwd is None:
         cpu = cpu_baseline(w, w.seed)
 
     if dist is not None:
@@ -456,7 +491,8 @@ def run_ours(args, w):
     if rank == 0:
         in_bytes = 4 * q.numel() * q.element_size() + lse.numel() * 4
         line = {
-            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "metric": METRIC if bwd is None else METRIC.replace("attention fwd", "attention bwd"),
+            "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * elapsed_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -467,7 +503,7 @@ def run_ours(args, w):
                               if in_bytes > L2_BYTES else "L2 not flushed (inputs < L2)")},
             "pct_of_peak": 100.0 * value / world / peak,
             "roofline": roofline,
-            "e2e": {"value": weak_scaling_value(w.flops, world, e2e_steps, e2e_s), "unit": "TFLOP/s",
+            "e2e": {"value": weak_scaling_value(flops, world, e2e_steps, e2e_s), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
             "clocks": clocks,
@@ -489,9 +525,10 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--path", default="fused", choices=["fused", "splitkv", "standard"],
+    ap.add_argument("--path", default="fused", choices=["fused", "splitkv", "standard", "backward"],
                     help="fused: fa_fwd; splitkv: fa_fwd_splitkv (key ranges + merge); "
-                         "standard: the materialising comparator (GEMM, softmax, GEMM)")
+                         "standard: the materialising comparator (GEMM, softmax, GEMM); "
+                         "backward: fa_bwd (dQ, dK, dV)")
     ap.add_argument("--splits", type=int, default=0, help="splitkv: key ranges (0 = default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-step-seconds", type=float, default=8.0,

@@ -3,7 +3,8 @@
     python -m exact_softmax_attention_02_b200.build [--force] [--verbose]
 
 The library is built from csrc/fa_fwd.cu (the fused forward, split-KV and
-merge) and csrc/standard_softmax.cu (the comparator's softmax), linked
+merge), csrc/fa_bwd.cu (the backward pass) and csrc/standard_softmax.cu (the
+comparator's softmax), linked
 against the static CUDA runtime; the driver entry point for tensor-map encoding is looked
 up at run time, so no libcuda link is needed.
 """
@@ -18,8 +19,9 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = [os.path.join(HERE, "csrc", "fa_fwd.cu"), os.path.join(HERE, "csrc", "standard_softmax.cu")]
-DEPENDS = SOURCES + [os.path.join(HERE, "csrc", "sm100.cuh"), os.path.join(ROOT, "include", "fa.h")]
+SOURCES = [os.path.join(HERE, "csrc", n) for n in ("fa_fwd.cu", "fa_bwd.cu", "standard_softmax.cu")]
+DEPENDS = SOURCES + [os.path.join(HERE, "csrc", "sm100.cuh"), os.path.join(HERE, "csrc", "host_util.h"),
+                     os.path.join(ROOT, "include", "fa.h")]
 OUTPUT = os.path.join(HERE, "libfa.so")
 
 NVCC_FLAGS = [

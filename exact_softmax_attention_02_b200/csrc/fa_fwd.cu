@@ -52,9 +52,13 @@
 #include <mutex>
 
 #include "fa.h"
+#include "host_util.h"
 #include "sm100.cuh"
 
 namespace fa {
+namespace bwd {
+cudaError_t read_and_clear_status(uint32_t* v);  // fa_bwd.cu
+}
 
 constexpr int kBM = 128;       // query rows per tile
 constexpr int kBN = 128;       // keys per tile
@@ -697,48 +701,21 @@ __global__ void __launch_bounds__(256)
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-namespace {
-
-thread_local char g_last_cuda_error[256] = "";
+namespace host {
+thread_local char g_last_error[256] = "";
 unsigned int g_debug_flags = 0;
 unsigned long long g_timeout_ns = 0;
-constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
+}  // namespace host
 
-fa_status cuda_fail(cudaError_t e, const char* what) {
-  snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", what, cudaGetErrorString(e));
-  return FA_ERR_CUDA;
-}
+namespace {
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
-}
-
-// [BH][N][d] bf16 viewed as a 3-D tensor (d fastest); boxes of 64 x box_rows
-// x 1 with the 128-byte swizzle.  Rows past N read as zero and are not stored.
-bool make_map(CUtensorMap* map, const void* base, int d, int N, int BH, int box_rows) {
-  auto enc = encode_tiled();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
-                        static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
-                           static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
+using host::cuda_fail;
+using host::g_debug_flags;
+using host::g_last_error;
+using host::g_timeout_ns;
+using host::kDefaultTimeoutNs;
+using host::make_map;
+using host::overlaps;
 
 struct DeviceInfo {
   bool checked = false;
@@ -768,7 +745,7 @@ fa_status launch(const void* Q, const void* K, const void* V, void* O, FwdParams
   CUtensorMap mq, mk, mv, mo;
   if (!make_map(&mq, Q, D, N, BH, kBM) || !make_map(&mk, K, D, N, BH, C::kKRows) ||
       !make_map(&mv, V, D, N, BH, kBM) || !make_map(&mo, O, D, N, BH, kBM)) {
-    snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed");
+    snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed");
     return FA_ERR_CUDA;
   }
   const long long rows_per_block = static_cast<long long>(kQTiles) * C::kRowsPerTile;
@@ -815,11 +792,6 @@ fa_status launch_merge(const float* o_part, const float* lse_part, void* O, floa
   return FA_OK;
 }
 
-bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
-  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
-  return x < y + nb && y < x + na;
-}
-
 }  // namespace
 }  // namespace fa
 
@@ -842,7 +814,7 @@ const char* fa_status_string(fa_status s) {
   return "unknown fa_status";
 }
 
-const char* fa_last_cuda_error(void) { return fa::g_last_cuda_error; }
+const char* fa_last_cuda_error(void) { return fa::g_last_error; }
 
 #ifdef FA_TRACE
 // Trace builds only: device buffer of kTraceCtas*4*kTraceIters*8 uint64 (or NULL).
@@ -1110,10 +1082,14 @@ fa_status fa_get_device_status_word(void* stream, unsigned int* word) {
   uint32_t v = 0;
   e = cudaMemcpyFromSymbol(&v, fa::g_device_status, sizeof(v));
   if (e != cudaSuccess) return fa::cuda_fail(e, "cudaMemcpyFromSymbol");
+  uint32_t vb = 0;
+  e = fa::bwd::read_and_clear_status(&vb);
+  if (e != cudaSuccess) return fa::cuda_fail(e, "backward status");
+  v |= vb;
   if (word) *word = v;
   if (v != 0) {
     const uint32_t zero = 0;
-    e = cudaMemcpyToSymbol(fa::g_device_status, &zero, sizeof(zero));
+    e = cudaMemcpyToSymbol(fa::g_device_status, &zero, sizeof(zero));  // backward's already cleared
     if (e != cudaSuccess) return fa::cuda_fail(e, "cudaMemcpyToSymbol");
     return FA_ERR_DEVICE_TIMEOUT;
   }

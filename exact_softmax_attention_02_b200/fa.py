@@ -66,6 +66,10 @@ def _load():
     lib.fa_fwd_splitkv_workspace_bytes.restype = ctypes.c_size_t
     lib.fa_fwd_splitkv_default_splits.argtypes = [c_int, c_int, c_int, c_int, c_int]
     lib.fa_fwd_splitkv_default_splits.restype = c_int
+    lib.fa_bwd.argtypes = [vp] * 10 + [ctypes.c_size_t, c_int, c_int, c_int, c_int, c_float, c_int, vp]
+    lib.fa_bwd.restype = c_int
+    lib.fa_bwd_workspace_bytes.argtypes = [c_int, c_int, c_int]
+    lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
     lib.fa_version.argtypes = []
     lib.fa_version.restype = ctypes.c_char_p
     _lib = lib
@@ -173,6 +177,33 @@ def fa_fwd_splitkv(q, k, v, o, lse=None, workspace=None, num_splits: int = 0,
                               workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                               B, H, N, d, float(scale), int(bool(causal)), int(num_splits),
                               _stream_handle(stream)))
+
+
+def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace=None, scale: float | None = None,
+           causal: bool = False, stream=None) -> None:
+    """Backward pass: dq, dk, dv of L = sum(o * do) for o = fa_fwd(q, k, v).
+
+    q, k, v, o, do, dq, dk, dv: CUDA bf16 [B, H, N, d] contiguous; lse: the
+    forward's fp32 [B, H, N].  ``workspace``: at least
+    fa_bwd_workspace_bytes(B, H, N) bytes of CUDA memory (allocated here if None).
+    """
+    lib = _load()
+    _check_qkvo(q, k, v, o)
+    _check_qkvo(do, dq, dk, dv)
+    if do.shape != q.shape:
+        raise ValueError("do, dq, dk, dv must have the shape of q")
+    B, H, N, d = q.shape
+    if lse.dtype != torch.float32 or not lse.is_cuda or tuple(lse.shape) != (B, H, N):
+        raise ValueError(f"lse must be a CUDA float32 [B, H, N] = {(B, H, N)} tensor")
+    need = int(lib.fa_bwd_workspace_bytes(B, H, N))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    _check(lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                      lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                      workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                      B, H, N, d, float(scale), int(bool(causal)), _stream_handle(stream)))
 
 
 def attention_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,

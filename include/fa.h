@@ -113,6 +113,32 @@ size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int N, int d, int causal, in
  * (1 for invalid arguments). */
 int fa_fwd_splitkv_default_splits(int B, int H, int N, int d, int causal);
 
+/*
+ * fa_bwd -- gradients of L = sum(O * dO) for O = fa_fwd(Q, K, V): dQ, dK, dV,
+ * recomputing the probabilities tile by tile from Q, K and the forward's LSE
+ * (lihaoran.work, "selected recomputation in the backward pass"; the
+ * derivative of the definition: dV = P^T dO, dS = P * (dO V^T - D) with
+ * D = rowsum(dO * O), dQ = scale dS K, dK = scale dS^T Q).
+ *
+ *   Q, K, V, O, dO  device, bf16 [B][H][N][d], read (O as written by fa_fwd).
+ *   LSE             device, fp32 [B][H][N], read (as written by fa_fwd).
+ *   dQ, dK, dV      device, bf16 [B][H][N][d], written.
+ *   workspace       device, 16-byte aligned, >= fa_bwd_workspace_bytes(B, H,
+ *                   N) bytes, overwritten (D, fp32 [B][H][N]).
+ *   B, H, N, d, scale, causal, stream: as for fa_fwd.
+ * The outputs and the workspace must not overlap the inputs or each other.
+ * Three kernels are enqueued on `stream`.  Errors as fa_fwd, plus
+ * FA_ERR_WORKSPACE for a short workspace; device-side give-ups are reported
+ * by fa_get_device_status().
+ */
+fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                 const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
+                 size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
+                 void* stream);
+
+/* Bytes of workspace fa_bwd needs (0 for invalid arguments). */
+size_t fa_bwd_workspace_bytes(int B, int H, int N);
+
 /* Size of the workspace built into the library for fa_fwd_splitkv_noalloc. */
 #define FA_NOALLOC_SCRATCH_BYTES (64 * 1024 * 1024)
 
@@ -171,7 +197,8 @@ const char* fa_status_string(fa_status status);
 
 /*
  * fa_get_device_status -- synchronise `stream`, then read and clear the
- * device status word of the current device.  Returns FA_ERR_DEVICE_TIMEOUT
+ * device status words (forward and backward kernels) of the current device.
+ * Returns FA_ERR_DEVICE_TIMEOUT
  * if any kernel launched by this library gave up on a bounded wait since the
  * last call (its outputs are then undefined), FA_ERR_CUDA if the
  * synchronisation failed, FA_OK otherwise.

@@ -151,3 +151,34 @@ def test_splitkv_default_splits(lib):
     assert lib.fa_fwd_splitkv_default_splits(4, 16, 4096, 64, 0) == 1
     # at least two key tiles per range
     assert lib.fa_fwd_splitkv_default_splits(1, 1, 512, 64, 0) == 2
+
+
+def test_bwd_argument_checks(lib):
+    vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.fa_bwd.argtypes = [vp] * 10 + [ctypes.c_size_t, ci, ci, ci, ci, cf, ci, vp]
+    lib.fa_bwd.restype = ci
+    lib.fa_bwd_workspace_bytes.argtypes = [ci, ci, ci]
+    lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
+    assert lib.fa_bwd_workspace_bytes(2, 3, 100) == 2 * 3 * 100 * 4
+    base = [A + k * 64 * MB for k in range(10)]  # Q K V O dO LSE dQ dK dV ws
+
+    def bwd(args=None, ws_bytes=1 << 20, N=128, d=64):
+        a = list(base if args is None else args)
+        return lib.fa_bwd(*a, ws_bytes, 1, 1, N, d, 0.125, 0, None)
+
+    for idx in range(10):
+        a = list(base)
+        a[idx] = None
+        assert bwd(a) == FA_ERR_NULL
+    assert bwd(d=96) == FA_ERR_UNSUPPORTED
+    assert bwd(N=0) == FA_ERR_SHAPE
+    assert bwd(ws_bytes=128 * 4 - 4) == FA_ERR_WORKSPACE
+    a = list(base)
+    a[6] = base[0] + 32  # dQ overlapping Q
+    assert bwd(a) == FA_ERR_ALIAS
+    a = list(base)
+    a[9] = base[6]  # workspace inside dQ
+    assert bwd(a) == FA_ERR_ALIAS
+    a = list(base)
+    a[7] = base[7] + 8
+    assert bwd(a) == FA_ERR_ALIGN
