@@ -17,10 +17,10 @@
 //                query tiles (tcgen05, A operands from TMEM).
 //   bwd_dq       one CTA per 128-query tile: S = Q K^T and dP = dO V^T, dS in
 //                place, dQ += dS K over the key tiles.
-// CTA layout of the two tiled kernels (256 threads): warp 0 TMA producer,
-// warp 1 TMEM owner and MMA issuer, warps 4-7 elementwise step and epilogue
-// (one thread per TMEM lane = one row of the tile).  Every wait is bounded
-// as in the forward kernel.
+// CTA layout of the two tiled kernels (384 threads): warp 0 TMA producer,
+// warp 1 TMEM owner and MMA issuer, warps 4-11 elementwise step and epilogue
+// (two threads per TMEM lane, i.e. per row of the tile, 64 columns each).
+// Every wait is bounded as in the forward kernel.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -39,8 +39,9 @@ namespace fa {
 namespace bwd {
 
 constexpr int kTile = 128;   // rows of a query tile, keys of a key tile
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr int kElemWarp0 = 4;
+constexpr int kElemThreads = 256;  // warps 4-11: two threads per row, 64 columns each
 constexpr uint32_t kTmemCols = 512;
 constexpr int kChunkBytes = kTile * 64 * 2;  // one 64-wide, 128-row swizzled box
 
@@ -61,9 +62,13 @@ struct BwdParams {
 __device__ uint32_t g_bwd_status;
 
 // TMEM column maps (both kernels): S or S^T at [0,128), dP or dP^T at
-// [128,256), accumulators from 256.  P / dS (bf16 pairs) overwrite the first
-// 64 columns of the tile they came from.
+// [128,256), accumulators from 256.  P / dS (bf16 pairs) overwrite their own
+// tile: the 32 values of columns 32c..32c+31 go, packed, to columns
+// 32c..32c+15, so each thread only overwrites what it has already read.
 constexpr uint32_t kColS = 0, kColDP = 128, kColAcc = 256;
+
+// TMEM column of the packed bf16 operand for K-step kk (16 keys or queries)
+__device__ __forceinline__ uint32_t packed_col(int kk) { return (kk >> 1) * 32 + (kk & 1) * 8; }
 
 // Work order shared by the tiled kernels: heads in groups, inside a group the
 // tiles with the most work first, cycling over the group's heads.
@@ -77,15 +82,16 @@ __device__ __forceinline__ void tile_of(const BwdParams& p, bool heavy_high, int
   *tile = heavy_high ? p.n_tiles - 1 - k : k;
 }
 
-// Elementwise step of one 128-column tile for the calling thread's row:
-// p = 2^(s * scale log2e - lse2), masked to 0 where `allowed` fails;
-// ds = p * (dp - dsub).  P (optional) and dS are written as bf16 pairs over
-// the first 64 columns of their own TMEM tiles, 32 columns at a time.
+// Elementwise step over 64 of the 128 columns (chunks c0, c0+1 of 32) of the
+// calling thread's row: p = 2^(s * scale log2e - lse2), masked to 0 where
+// `allowed` fails; ds = p * (dp - dsub).  P (optional) and dS are written as
+// bf16 pairs into the first half of each chunk's own columns.
 template <bool WRITE_P, typename ColLse, typename ColDsub, typename Allowed>
-__device__ __forceinline__ void p_ds_tile(uint32_t tS, uint32_t tDP, float sl2, ColLse col_lse2,
+__device__ __forceinline__ void p_ds_tile(uint32_t tS, uint32_t tDP, int c0, float sl2, ColLse col_lse2,
                                           ColDsub col_dsub, Allowed allowed) {
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
+  for (int cc = 0; cc < 2; ++cc) {
+    const int c = c0 + cc;
     uint32_t s[32], dp[32];
     tmem_ld32(tS + c * 32, s);
     tmem_ld32(tDP + c * 32, dp);
@@ -103,17 +109,20 @@ __device__ __forceinline__ void p_ds_tile(uint32_t tS, uint32_t tDP, float sl2, 
       pk[e >> 1] = pack_bf16x2(p0, p1);
       dk[e >> 1] = pack_bf16x2(d0, d1);
     }
-    if (WRITE_P) tmem_st16(tS + c * 16, pk);
-    tmem_st16(tDP + c * 16, dk);
+    if (WRITE_P) tmem_st16(tS + c * 32, pk);
+    tmem_st16(tDP + c * 32, dk);
   }
 }
 
-// Store one 128 x D tile held in TMEM (this thread's row r, fp32) as bf16 via
-// the 128-byte-swizzled staging buffer and a TMA store.
+// Store 32-column chunks [cb, ce) of a 128 x D tile held in TMEM (this
+// thread's row r, fp32) as bf16 into the 128-byte-swizzled staging buffer
+// that a TMA store then writes out.
 template <int D>
-__device__ __forceinline__ void store_tile(uint32_t tAcc, float mul, uint8_t* stage, int r) {
+__device__ __forceinline__ void store_tile(uint32_t tAcc, float mul, uint8_t* stage, int r, int cb,
+                                           int ce) {
 #pragma unroll
   for (int c = 0; c < D / 32; ++c) {
+    if (c < cb || c >= ce) continue;
     uint32_t o[32];
     tmem_ld32(tAcc + c * 32, o);
     tmem_wait_ld();
@@ -213,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&st_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(ds_ready, kTile);
+    mbar_init(ds_ready, kElemThreads);
     mbar_init(acc_done, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -276,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_acc = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b, bool accumulate) {
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk) {
-          mma_ts(d_tmem, a_tmem + kk * 8, sw128_desc(b + kk * 2048, kChunkBytes, 1024), idAcc,
+          mma_ts(d_tmem, a_tmem + packed_col(kk), sw128_desc(b + kk * 2048, kChunkBytes, 1024), idAcc,
                  (accumulate || kk > 0) ? 1u : 0u);
         }
       };
@@ -300,6 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_drain(mma_done, 0, tmo);
     }
   } else if (warp >= kElemWarp0) {
+    const int half = (warp - kElemWarp0) >> 2;  // which 64 of the 128 query columns
     const int wq = warp & 3;
     const int r = wq * 32 + lane;  // key row inside the tile
     const int key = j * kTile + r;
@@ -308,23 +318,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = p.scale_log2;
     const float* lse_g = p.lse + static_cast<size_t>(bh) * p.N;
     const float* d_g = p.dd + static_cast<size_t>(bh) * p.N;
-    // LSE (log2 units) and D of the 128 queries of a tile, staged in shared
-    // memory (two buffers); queries past N get LSE = +inf, so P = 0 there.
-    auto fetch = [&](int i, float& l2, float& dv) {
+    // LSE (log2 units; first half of the threads) and D (second half) of the
+    // 128 queries of a tile, staged in shared memory (two buffers); queries
+    // past N get LSE = +inf, so P = 0 there.
+    auto fetch = [&](int i) {
       const int qi = i * kTile + r;
-      l2 = qi < p.N ? lse_g[qi] * 1.4426950408889634f : INFINITY;
-      dv = qi < p.N ? d_g[qi] : 0.f;
+      if (half == 0) return qi < p.N ? lse_g[qi] * 1.4426950408889634f : INFINITY;
+      return qi < p.N ? d_g[qi] : 0.f;
     };
-    float l2n = 0.f, dvn = 0.f;
-    if (n_iter > 0) fetch(i_first, l2n, dvn);
-    sLse[r] = l2n;
-    sD[r] = dvn;
-    named_bar_sync(1, kTile);
+    float* stage_buf = half == 0 ? sLse : sD;
+    float nxt = n_iter > 0 ? fetch(i_first) : 0.f;
+    stage_buf[r] = nxt;
+    named_bar_sync(1, kElemThreads);
     bool ok = true;
     for (int it = 0; it < n_iter; ++it) {
       const int i = i_first + it;
       const int buf = it & 1;
-      if (it + 1 < n_iter) fetch(i + 1, l2n, dvn);  // next tile's, early
+      if (it + 1 < n_iter) nxt = fetch(i + 1);  // next tile's, early
       const bool good = __all_sync(
           0xffffffffu, mbar_wait(s_full, static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteS));
       if (good) {
@@ -333,31 +343,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float* dt = sD + buf * kTile;
         const bool diag = CAUSAL && i == j;
         p_ds_tile<true>(
-            tS, tDP, sl2, [&](int c) { return lt[c]; }, [&](int c) { return dt[c]; },
+            tS, tDP, 2 * half, sl2, [&](int c) { return lt[c]; }, [&](int c) { return dt[c]; },
             [&](int c) { return !diag || i * kTile + c >= key; });
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(ds_ready);
       }
-      sLse[(buf ^ 1) * kTile + r] = l2n;
-      sD[(buf ^ 1) * kTile + r] = dvn;
+      stage_buf[(buf ^ 1) * kTile + r] = nxt;
       // one barrier per iteration for every thread: it publishes the next
       // tile's LSE/D and makes a give-up decision uniform across the warps
-      if (named_bar_or(1, kTile, !good)) {
+      if (named_bar_or(1, kElemThreads, !good)) {
         ok = false;
         break;
       }
     }
     if (ok) ok = mbar_wait(acc_done, 0, abort_flag, status, tmo, kSiteO);
-    const bool failed = named_bar_or(2, kTile, !ok);
+    const bool failed = named_bar_or(2, kElemThreads, !ok);
     if (!failed && n_iter > 0) {
       tc_fence_after();
-      // K and V are no longer read by any MMA: they stage dK and dV
-      store_tile<D>(tmem + lane_base + kColAcc + D, p.scale, sK, r);
-      store_tile<D>(tmem + lane_base + kColAcc, 1.f, sV, r);
+      // K and V are no longer read by any MMA: they stage dK (first half of
+      // the threads) and dV (second half)
+      if (half == 0)
+        store_tile<D>(tmem + lane_base + kColAcc + D, p.scale, sK, r, 0, D / 32);
+      else
+        store_tile<D>(tmem + lane_base + kColAcc, 1.f, sV, r, 0, D / 32);
       fence_proxy_async_smem();
-      named_bar_sync(1, kTile);
-      if (r == 0) {
+      named_bar_sync(1, kElemThreads);
+      if (half == 0 && r == 0) {
         for (int c = 0; c < C::kChunks; ++c) {
           tma_store_3d(&tmdK, sK + c * kChunkBytes, c * 64, j * kTile, bh);
           tma_store_3d(&tmdV, sV + c * kChunkBytes, c * 64, j * kTile, bh);
@@ -430,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&st_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(ds_ready, kTile);
+    mbar_init(ds_ready, kElemThreads);
     mbar_init(acc_done, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -502,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // dQ += dS K: A = dS in TMEM (over dP), B = K tile as [keys][d] (MN-major)
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk) {
-          mma_ts(tmem + kColAcc, tmem + kColDP + kk * 8, sw128_desc(k + kk * 2048, kChunkBytes, 1024),
+          mma_ts(tmem + kColAcc, tmem + kColDP + packed_col(kk), sw128_desc(k + kk * 2048, kChunkBytes, 1024),
                  idAcc, (it > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&st_empty[s]);
@@ -512,6 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_drain(mma_done, 0, tmo);
     }
   } else if (warp >= kElemWarp0) {
+    const int half = (warp - kElemWarp0) >> 2;  // which 64 of the 128 key columns
     const int wq = warp & 3;
     const int r = wq * 32 + lane;  // query row inside the tile
     const int row = i * kTile + r;
@@ -531,20 +544,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int kbase = it * kTile;
       const bool masked = (kbase + kTile > p.N) || (CAUSAL && kbase + kTile - 1 > i * kTile);
       p_ds_tile<false>(
-          tS, tDP, sl2, [&](int) { return lse2; }, [&](int) { return dsub; },
+          tS, tDP, 2 * half, sl2, [&](int) { return lse2; }, [&](int) { return dsub; },
           [&](int c) { return !masked || kbase + c <= key_limit; });
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(ds_ready);
     }
     if (ok) ok = mbar_wait(acc_done, 0, abort_flag, status, tmo, kSiteO);
-    const bool failed = named_bar_or(2, kTile, !ok);
+    const bool failed = named_bar_or(2, kElemThreads, !ok);
     if (!failed) {
       tc_fence_after();
-      store_tile<D>(tmem + lane_base + kColAcc, p.scale, sQ, r);  // Q no longer read
+      // Q is no longer read by any MMA: it stages dQ, each half of the
+      // threads taking half of the columns
+      store_tile<D>(tmem + lane_base + kColAcc, p.scale, sQ, r, half * (D / 64), (half + 1) * (D / 64));
       fence_proxy_async_smem();
-      named_bar_sync(1, kTile);
-      if (r == 0) {
+      named_bar_sync(1, kElemThreads);
+      if (half == 0 && r == 0) {
         for (int c = 0; c < C::kChunks; ++c) tma_store_3d(&tmdQ, sQ + c * kChunkBytes, c * 64, i * kTile, bh);
         bulk_commit_group();
         bulk_wait_group_read0();
