@@ -10,6 +10,8 @@ from .attention import (  # noqa: F401
     attention_backward,
     attention_full,
     attention_rows,
+    block_layout_from_csr,
+    block_sparse_attention_rows,
     brute_force_attention,
     flops_for_rows,
     merge_block,

@@ -45,6 +45,9 @@ Three functions, three independent computations:
 ``attention_backward`` gives dQ, dK, dV of L = sum(O * dO), the derivative
 of the same definition (pinned by finite differences).
 
+``block_sparse_attention_rows`` restricts the allowed keys to the blocks a
+block layout retains (the block-sparse comparison the pages suggest).
+
 ``attention_rows(..., key_range=(lo, hi))`` gives the partial state of one
 key range, and ``merge_states`` folds such states together (the block update
 applied to whole states); merged states over disjoint ranges equal the full
@@ -68,6 +71,8 @@ __all__ = [
     "attention_backward",
     "merge_states",
     "attention_full",
+    "block_sparse_attention_rows",
+    "block_layout_from_csr",
     "online_attention_rows",
     "merge_block",
     "brute_force_attention",
@@ -100,7 +105,7 @@ def _group_rows(rows: np.ndarray):
         yield b, h, pos, rows[pos, 2]
 
 
-def attention_rows(q, k, v, scale: float, causal: bool, rows, key_range=None):
+def attention_rows(q, k, v, scale: float, causal: bool, rows, key_range=None, key_mask=None):
     """Exact attention output and LSE for the selected rows.
 
     Follows the dense definition O = softmax(scale * Q K^T) V
@@ -117,6 +122,8 @@ def attention_rows(q, k, v, scale: float, causal: bool, rows, key_range=None):
       key_range: optional (lo, hi): only keys lo <= j < hi are allowed (the
                partial state of one key range).  A row with no allowed key
                gets O = 0 and LSE = -inf (the empty state, weight 0 in a merge).
+      key_mask: optional callable (b, h, i [r], j [N]) -> bool [r, N]; keys
+               where it is false are not allowed (block-sparse retention).
 
     Returns:
       (O, LSE): float64 arrays [R, d] and [R].
@@ -141,6 +148,8 @@ def attention_rows(q, k, v, scale: float, causal: bool, rows, key_range=None):
             if key_range is not None:
                 lo, hi = key_range
                 s = np.where((j[None, :] >= lo) & (j[None, :] < hi), s, -np.inf)
+            if key_mask is not None:
+                s = np.where(key_mask(b, h, i, j), s, -np.inf)
             m = s.max(axis=1)  # largest score of each row
             empty = np.isneginf(m)
             m_safe = np.where(empty, 0.0, m)
@@ -159,6 +168,47 @@ def attention_full(q, k, v, scale: float, causal: bool):
     rows = np.stack([b.ravel(), h.ravel(), i.ravel()], axis=1)
     o, l = attention_rows(q, k, v, scale, causal, rows)
     return o.reshape(B, H, N, d), l.reshape(B, H, N)
+
+
+def block_sparse_attention_rows(q, k, v, scale: float, causal: bool, rows, layout,
+                                block_q: int, block_k: int):
+    """Attention restricted to the key blocks a block layout retains.
+
+    The pages treat sparsity as a separate design dimension that decides which
+    query-key interactions are kept (liminalml.com "FlashAttention", the
+    question "Is it sparse attention?"), and suggest comparing exact and
+    block-sparse attention at matched output error (interactiveml.org
+    "FlashAttention saves the matrix, not the quadratic work", the suggested
+    experiments).  Reading: block-sparse attention is the same softmax over a
+    smaller allowed set.  Query i may see key j only if
+    layout[i // block_q, j // block_k] is set (and j <= i when causal).  A
+    query with no allowed key gets O = 0 and LSE = -inf.
+
+    Args:
+      layout: bool array [ceil(N / block_q), ceil(N / block_k)], shared by
+              every (b, h).
+      block_q, block_k: query rows and keys per block.
+    Other arguments and the return value as in ``attention_rows``.
+    """
+    lay = np.asarray(layout, dtype=bool)
+
+    def mask(b, h, i, j):
+        return lay[np.asarray(i)[:, None] // block_q, np.asarray(j)[None, :] // block_k]
+
+    return attention_rows(q, k, v, scale, causal, rows, key_mask=mask)
+
+
+def block_layout_from_csr(row_ptr, col_idx, n_kblocks: int) -> np.ndarray:
+    """Dense bool layout [len(row_ptr) - 1, n_kblocks] from CSR block lists.
+
+    Row r retains key blocks col_idx[row_ptr[r]:row_ptr[r+1]].
+    """
+    row_ptr = np.asarray(row_ptr, dtype=np.int64)
+    col_idx = np.asarray(col_idx, dtype=np.int64)
+    lay = np.zeros((len(row_ptr) - 1, n_kblocks), dtype=bool)
+    for r in range(len(row_ptr) - 1):
+        lay[r, col_idx[row_ptr[r]:row_ptr[r + 1]]] = True
+    return lay
 
 
 def merge_block(m, total, acc, scores, values):
@@ -297,13 +347,16 @@ def online_attention_rows(q, k, v, scale: float, causal: bool, rows, tile: int =
     return out, lse
 
 
-def brute_force_attention(q, k, v, scale: float, causal: bool):
+def brute_force_attention(q, k, v, scale: float, causal: bool, layout=None, block_q: int = 1,
+                          block_k: int = 1):
     """Pure-Python softmax attention without max subtraction (tiny inputs).
 
     O_i = sum_j e^{s_ij} V_j / sum_j e^{s_ij}, summed exactly with
     math.fsum; LSE_i = ln sum_j e^{s_ij}.  Only valid while every e^{s}
-    is representable, i.e. for small scores.  Returns nested lists
-    O[b][h][i][c] and LSE[b][h][i].
+    is representable, i.e. for small scores.  With a block layout (nested
+    lists or array of booleans), key j is skipped for query i unless
+    layout[i // block_q][j // block_k] is set; a query left with no key gets
+    O = 0 and LSE = -inf.  Returns nested lists O[b][h][i][c] and LSE[b][h][i].
     """
     B, H, N, d = (int(x) for x in np.shape(q))
     qf, kf, vf = (np.asarray(t, dtype=np.float64).tolist() for t in (q, k, v))
@@ -316,8 +369,13 @@ def brute_force_attention(q, k, v, scale: float, causal: bool):
                 for j in range(N):
                     if causal and j > i:
                         continue
+                    if layout is not None and not layout[i // block_q][j // block_k]:
+                        continue
                     s = scale * math.fsum(qf[b][h][i][c] * kf[b][h][j][c] for c in range(d))
                     e.append((j, math.exp(s)))
+                if not e:
+                    L[b][h][i] = -math.inf
+                    continue
                 z = math.fsum(w for _, w in e)
                 for c in range(d):
                     O[b][h][i][c] = math.fsum(w * vf[b][h][j][c] for j, w in e) / z

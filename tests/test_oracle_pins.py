@@ -519,3 +519,100 @@ def test_backward_pins_reject_a_dropped_term():
     num = (_loss(qp, k, v, do, 1.0, False) - _loss(qm, k, v, do, 1.0, False)) / (2 * eps)
     assert abs(dq[0, 0, 2, 1] - num) < 1e-7
     assert abs(bad_dq[2, 1] - num) > 1e-3
+
+
+# ---------------------------------------------------------------------------
+# Block-sparse attention: the softmax over the key blocks a layout retains
+# ---------------------------------------------------------------------------
+
+def _random_layout(rng, nqb, nkb, density=0.5):
+    lay = rng.random((nqb, nkb)) < density
+    lay[0, :] = False  # one query block with no key at all
+    return lay
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_block_sparse_brute_force_tiny(seed):
+    """Random block layouts (one row block empty) against pure-Python loops."""
+    from oracle import block_sparse_attention_rows
+
+    rng = np.random.default_rng(300 + seed)
+    B, H = int(rng.integers(1, 3)), int(rng.integers(1, 3))
+    N, d = int(rng.integers(5, 18)), int(rng.integers(1, 6))
+    bq, bk = int(rng.integers(1, 5)), int(rng.integers(1, 5))
+    lay = _random_layout(rng, -(-N // bq), -(-N // bk))
+    q = rng.standard_normal((B, H, N, d))
+    k = rng.standard_normal((B, H, N, d))
+    v = rng.standard_normal((B, H, N, d))
+    causal = bool(seed % 2)
+    bo, bl = brute_force_attention(q, k, v, 0.7, causal, layout=lay, block_q=bq, block_k=bk)
+    o, l = block_sparse_attention_rows(q, k, v, 0.7, causal, all_rows(B, H, N), lay, bq, bk)
+    assert np.allclose(o, np.array(bo).reshape(o.shape), rtol=1e-12, atol=1e-13)
+    bl = np.array(bl).reshape(l.shape)
+    assert (np.isneginf(l) == np.isneginf(bl)).all()
+    fin = np.isfinite(bl)
+    assert np.allclose(l[fin], bl[fin], rtol=1e-12, atol=1e-13)
+    # the empty first query block: O = 0, LSE = -inf
+    first = all_rows(B, H, N)[:, 2] < bq
+    assert (o[first] == 0).all() and np.isneginf(l[first]).all()
+
+
+def test_block_sparse_full_layout_is_dense_and_block_diagonal_is_per_block():
+    """All blocks retained = dense attention; a block-diagonal layout = each block alone."""
+    from oracle import block_sparse_attention_rows
+
+    rng = np.random.default_rng(21)
+    B, H, N, d = 1, 2, 96, 8
+    q, k, v = (rng.standard_normal((B, H, N, d)) for _ in range(3))
+    rows = all_rows(B, H, N)
+    dense_o, dense_l = attention_rows(q, k, v, 0.5, True, rows)
+    o, l = block_sparse_attention_rows(q, k, v, 0.5, True, rows, np.ones((3, 6), bool), 32, 16)
+    assert np.allclose(o, dense_o, rtol=1e-13, atol=1e-14) and np.allclose(l, dense_l, rtol=1e-13)
+    # block-diagonal with 32-row and 32-key blocks: three independent problems
+    o, l = block_sparse_attention_rows(q, k, v, 0.5, False, rows, np.eye(3, dtype=bool), 32, 32)
+    o = o.reshape(B, H, N, d)
+    l = l.reshape(B, H, N)
+    for blk in range(3):
+        sl = slice(32 * blk, 32 * blk + 32)
+        bo, bl = attention_full(q[:, :, sl], k[:, :, sl], v[:, :, sl], 0.5, False)
+        assert np.allclose(o[:, :, sl], bo, rtol=1e-12, atol=1e-13)
+        assert np.allclose(l[:, :, sl], bl, rtol=1e-12, atol=1e-13)
+
+
+def test_block_sparse_single_block_closed_form():
+    """One retained key block whose values all equal c: O = c, LSE = logsumexp of its scores."""
+    from oracle import block_sparse_attention_rows
+
+    N, d = 12, 3
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal((1, 1, N, d))
+    k = rng.standard_normal((1, 1, N, d))
+    v = rng.standard_normal((1, 1, N, d))
+    v[0, 0, 4:8] = [1.5, -2.0, 0.25]
+    lay = np.zeros((3, 3), bool)
+    lay[:, 1] = True  # keys 4..7 only
+    o, l = block_sparse_attention_rows(q, k, v, 1.0, False, all_rows(1, 1, N), lay, 4, 4)
+    assert np.allclose(o, [1.5, -2.0, 0.25], rtol=1e-14)
+    s = q[0, 0] @ k[0, 0, 4:8].T
+    assert np.allclose(l, np.log(np.exp(s).sum(axis=1)), rtol=1e-13)
+
+
+def test_block_sparse_pins_reject_a_transposed_layout():
+    """A mutant that indexes the layout as [key block, query block] fails the brute-force pin."""
+    rng = np.random.default_rng(77)
+    N, d, bq, bk = 12, 2, 3, 4
+    lay = np.zeros((4, 3), bool)
+    lay[3, 0] = lay[1, 2] = lay[0, 0] = lay[2, 1] = True
+    q, k, v = (rng.standard_normal((1, 1, N, d)) for _ in range(3))
+    lay_t = lambda b, h, i, j: lay.T[np.minimum(np.asarray(i)[:, None] // bk, 2),
+                                     np.minimum(np.asarray(j)[None, :] // bq, 3)]
+    bad_o, _ = attention_rows(q, k, v, 1.0, False, all_rows(1, 1, N), key_mask=lay_t)
+    bo, _ = brute_force_attention(q, k, v, 1.0, False, layout=lay, block_q=bq, block_k=bk)
+    assert not np.allclose(bad_o, np.array(bo).reshape(bad_o.shape), atol=1e-6)
+
+
+def test_block_layout_from_csr():
+    from oracle import block_layout_from_csr
+
+    lay = block_layout_from_csr([0, 2, 2, 3], [0, 3, 1], 4)
+    assert lay.tolist() == [[True, False, False, True], [False] * 4, [False, True, False, False]]
