@@ -63,6 +63,8 @@ cudaError_t read_and_clear_status(uint32_t* v);  // fa_bwd.cu
 constexpr int kBM = 128;       // query rows per tile
 constexpr int kBN = 128;       // keys per tile
 constexpr int kQTiles = 2;     // query tiles per CTA
+static_assert(FA_BLOCK_Q == kQTiles * kBM && FA_BLOCK_K == kBN,
+              "a block-sparse block is one CTA's query rows by one key tile");
 constexpr int kThreads = 384;  // 12 warps
 constexpr int kSoftmaxWarp0 = 4;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -104,6 +106,11 @@ struct FwdParams {
   int kv_per_split;
   float* o_part;    // [num_splits][BH][N][d]
   float* lse_part;  // [num_splits][BH][N]
+  // block-sparse only: the key tiles each 256-row query block retains, as
+  // CSR lists (strictly ascending within a block), shared by every head
+  const int* blk_row_ptr;  // [n_qblk + 1]
+  const int* blk_col_idx;  // [blk_nnz]
+  int blk_nnz;
 };
 
 __device__ uint32_t g_device_status;
@@ -151,7 +158,7 @@ struct Cfg {
 // B and loads half of every K/V tile.  Each CTA's TMA signals a local barrier;
 // a forwarding warp then arrives on the even CTA's barrier, so that both CTAs
 // can drain their own copies exactly if they have to unwind.
-template <int D, bool CAUSAL, bool PAIR, bool SPLIT>
+template <int D, bool CAUSAL, bool PAIR, bool SPLIT, bool SPARSE>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -162,6 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int SB = C::kStageBytes;
   static_assert(!PAIR || D == 128, "the pair kernel splits d = 128 into two 64-wide halves");
   static_assert(!(PAIR && SPLIT), "split-KV uses the single-CTA shape");
+  static_assert(!(SPARSE && (PAIR || SPLIT)), "block-sparse uses the single-CTA, unsplit shape");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -214,11 +222,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   // from kv_end-1 down to kv_lo
   const int kv_lo = SPLIT ? split * p.kv_per_split : 0;
   const int kv_end = SPLIT ? min(j_last[1] + 1, kv_lo + p.kv_per_split) : j_last[1] + 1;
-  const int n_iter = max(0, kv_end - kv_lo);
+  int n_iter = max(0, kv_end - kv_lo);
   // iterations before a query tile's first unmasked key tile are skipped for
   // it; a tile whose first iteration is past n_iter has no keys in this range
-  const int first_it[2] = {kv_end - 1 - min(j_last[0], kv_end - 1), 0};
+  int first_it[2] = {kv_end - 1 - min(j_last[0], kv_end - 1), 0};
+  // Block-sparse: this block's retained key tiles, visited from the last
+  // entry down.  Entries past tile 1's diagonal are seen by no row and are
+  // dropped; leading visits past tile 0's diagonal are skipped for tile 0.
+  // A malformed list raises kStatusLayout; out-of-range or out-of-order
+  // entries are then masked out entirely (no memory outside the tensors is
+  // touched), and the outputs are not meaningful.
+  const int* blk = nullptr;
+  if (SPARSE) {
+    int beg = __ldg(p.blk_row_ptr + qblk), end = __ldg(p.blk_row_ptr + qblk + 1);
+    if (!(0 <= beg && beg <= end && end <= p.blk_nnz)) {
+      if (threadIdx.x == 0) atomicOr(&g_device_status, kStatusLayout);
+      beg = end = 0;
+    }
+    blk = p.blk_col_idx + beg;
+    int n = end - beg;
+    while (n > 0 && __ldg(blk + n - 1) > j_last[1]) {
+      if (threadIdx.x == 0 && __ldg(blk + n - 1) >= p.n_kv) atomicOr(&g_device_status, kStatusLayout);
+      --n;
+    }
+    int skip = 0;
+    while (skip < n && __ldg(blk + n - 1 - skip) > j_last[0]) ++skip;
+    n_iter = n;
+    first_it[0] = skip;
+  }
   const bool tile_active[2] = {first_it[0] < n_iter, n_iter > 0};
+  // key tile of iteration it
+  auto kv_tile = [&](int it) { return SPARSE ? __ldg(blk + n_iter - 1 - it) : kv_end - 1 - it; };
   const uint64_t tmo = p.timeout_ns;
 
   if (threadIdx.x == 0) {
@@ -274,7 +308,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int i = 0;  // loads issued into the ring, in consumption order K0 V0 K1 V1 ...
       for (int it = 0; it < n_iter && ok; ++it) {
-        const int j = kv_end - 1 - it;
+        // (a block-sparse entry out of range is loaded clamped and masked)
+        const int j = SPARSE ? min(max(kv_tile(it), 0), p.n_kv - 1) : kv_tile(it);
         for (int kv = 0; kv < 2; ++kv) {
           const int s = i % S;
           const uint32_t ph = static_cast<uint32_t>(i / S) & 1u;
@@ -468,7 +503,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int it = first_it[t]; it < n_iter && ok; ++it) {
       const int li = it - first_it[t];
-      const int j = kv_end - 1 - it;
+      int j = kv_tile(it);
+      // a block-sparse entry out of range or out of order contributes nothing
+      bool bad = false;
+      if (SPARSE) {
+        bad = j < 0 || j >= p.n_kv || (it > 0 && j >= kv_tile(it - 1));
+        if (bad) {
+          if ((threadIdx.x & 127) == 0) atomicOr(&g_device_status, kStatusLayout);
+          j = 0;
+        }
+      }
       ok = __all_sync(0xffffffffu,
                       mbar_wait<PAIR>(&s_full[t], static_cast<uint32_t>(li) & 1u, abort_flag, status, tmo, kSiteS));
       if (!ok) break;
@@ -482,13 +526,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tr) FA_TRACE_MARK(1 + t, it, 1);
 
       const int kbase = j * kBN;
-      const bool masked = (kbase + kBN > p.N) || (CAUSAL && kbase + kBN - 1 > row0);
+      const bool masked = bad || (kbase + kBN > p.N) || (CAUSAL && kbase + kBN - 1 > row0);
       if (masked) {
+        const int lim = bad ? -1 : key_limit;
 #pragma unroll
         for (int q = 0; q < 4; ++q)
 #pragma unroll
           for (int c = 0; c < 32; ++c)
-            if (kbase + q * 32 + c > key_limit) sr[q][c] = __float_as_uint(-INFINITY);
+            if (kbase + q * 32 + c > lim) sr[q][c] = __float_as_uint(-INFINITY);
       }
       // row maximum of the raw scores (scale > 0 keeps the argmax): eight
       // independent chains of three-input maxima
@@ -612,8 +657,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(tO + c * 32, o);
-        tmem_wait_ld();
+        if (tile_active[t]) {
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld();
+        } else {  // no retained key (block-sparse): O = 0
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = 0u;
+        }
         uint8_t* rowp = stage + (c >> 1) * kChunkBytes + r * 128;
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
@@ -720,7 +770,7 @@ using host::overlaps;
 struct DeviceInfo {
   bool checked = false;
   bool sm100 = false;
-  bool attr_set[16] = {};
+  bool attr_set[32] = {};
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_devices[kMaxDevices];
@@ -737,10 +787,10 @@ template <int D>
 constexpr bool kUsePair = false;
 #endif
 
-template <int D, bool CAUSAL, bool SPLIT>
+template <int D, bool CAUSAL, bool SPLIT, bool SPARSE = false>
 fa_status launch(const void* Q, const void* K, const void* V, void* O, FwdParams prm, int N, int BH,
                  cudaStream_t stream, DeviceInfo& dev) {
-  constexpr bool PAIR = kUsePair<D> && !SPLIT;
+  constexpr bool PAIR = kUsePair<D> && !SPLIT && !SPARSE;
   using C = Cfg<D, PAIR>;
   CUtensorMap mq, mk, mv, mo;
   if (!make_map(&mq, Q, D, N, BH, kBM) || !make_map(&mk, K, D, N, BH, C::kKRows) ||
@@ -753,8 +803,9 @@ fa_status launch(const void* Q, const void* K, const void* V, void* O, FwdParams
   const long long units = static_cast<long long>(BH) * prm.n_qblk;
   const long long grid = units * (SPLIT ? prm.num_splits : (PAIR ? 2 : 1));
   if (grid > 0x7fffffffll) return FA_ERR_SHAPE;
-  constexpr int slot = (D == 128 ? 8 : 0) + (CAUSAL ? 4 : 0) + (PAIR ? 2 : 0) + (SPLIT ? 1 : 0);
-  auto kern = fa_fwd_kernel<D, CAUSAL, PAIR, SPLIT>;
+  constexpr int slot =
+      (SPARSE ? 16 : 0) + (D == 128 ? 8 : 0) + (CAUSAL ? 4 : 0) + (PAIR ? 2 : 0) + (SPLIT ? 1 : 0);
+  auto kern = fa_fwd_kernel<D, CAUSAL, PAIR, SPLIT, SPARSE>;
   if (!dev.attr_set[slot]) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -810,6 +861,7 @@ const char* fa_status_string(fa_status s) {
     case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT: a kernel gave up on a bounded wait";
     case FA_ERR_ALIAS: return "FA_ERR_ALIAS: O, LSE or the workspace overlaps an input or each other";
     case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: the workspace is smaller than required";
+    case FA_ERR_LAYOUT: return "FA_ERR_LAYOUT: a block-sparse list was out of range or out of order";
   }
   return "unknown fa_status";
 }
@@ -1011,6 +1063,41 @@ fa_status fa_fwd_splitkv(const void* Q, const void* K, const void* V, void* O, f
                   : launch_merge<64>(prm.o_part, prm.lse_part, O, LSE, rows, num_splits, st);
 }
 
+fa_status fa_fwd_block_sparse(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                              const int* block_row_ptr, const int* block_col_idx, int nnz, int B,
+                              int H, int N, int d, float scale, int causal, void* stream) {
+  using namespace fa;
+  FwdParams prm;
+  DeviceInfo* dev = nullptr;
+  fa_status st0 = check_args(Q, K, V, O, LSE, B, H, N, d, scale);
+  if (st0 != FA_OK) return st0;
+  if (block_row_ptr == nullptr || (nnz > 0 && block_col_idx == nullptr)) return FA_ERR_NULL;
+  if (nnz < 0) return FA_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(block_row_ptr) & 3u) || (reinterpret_cast<uintptr_t>(block_col_idx) & 3u))
+    return FA_ERR_ALIGN;
+  const size_t n_blocks = static_cast<size_t>((N + FA_BLOCK_Q - 1) / FA_BLOCK_Q);
+  const size_t rp_bytes = (n_blocks + 1) * 4, ci_bytes = static_cast<size_t>(nnz) * 4;
+  const size_t nbytes = static_cast<size_t>(B) * H * N * d * 2;
+  const size_t lbytes = static_cast<size_t>(B) * H * N * 4;
+  if (overlaps(O, nbytes, block_row_ptr, rp_bytes) || (nnz > 0 && overlaps(O, nbytes, block_col_idx, ci_bytes)) ||
+      (LSE && (overlaps(LSE, lbytes, block_row_ptr, rp_bytes) ||
+               (nnz > 0 && overlaps(LSE, lbytes, block_col_idx, ci_bytes)))))
+    return FA_ERR_ALIAS;
+  st0 = prepare(LSE, B, H, N, d, scale, &prm, &dev);
+  if (st0 != FA_OK) return st0;
+  prm.blk_row_ptr = block_row_ptr;
+  prm.blk_col_idx = block_col_idx;
+  prm.blk_nnz = nnz;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int bh = prm.BH;
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  if (d == 128)
+    return causal ? launch<128, true, false, true>(Q, K, V, O, prm, N, bh, st, *dev)
+                  : launch<128, false, false, true>(Q, K, V, O, prm, N, bh, st, *dev);
+  return causal ? launch<64, true, false, true>(Q, K, V, O, prm, N, bh, st, *dev)
+                : launch<64, false, false, true>(Q, K, V, O, prm, N, bh, st, *dev);
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------
@@ -1091,7 +1178,7 @@ fa_status fa_get_device_status_word(void* stream, unsigned int* word) {
     const uint32_t zero = 0;
     e = cudaMemcpyToSymbol(fa::g_device_status, &zero, sizeof(zero));  // backward's already cleared
     if (e != cudaSuccess) return fa::cuda_fail(e, "cudaMemcpyToSymbol");
-    return FA_ERR_DEVICE_TIMEOUT;
+    return (v & fa::kStatusTimeout) ? FA_ERR_DEVICE_TIMEOUT : FA_ERR_LAYOUT;
   }
   return FA_OK;
 }

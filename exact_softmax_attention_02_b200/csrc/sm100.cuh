@@ -72,6 +72,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Status bits a kernel may raise in its device status word.
 enum : uint32_t {
   kStatusTimeout = 1u,  // a bounded wait gave up
+  kStatusLayout = 2u,   // a block-sparse list was malformed
 };
 
 // Wait until the phase with the given parity has completed.  Gives up (and

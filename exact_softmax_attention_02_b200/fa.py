@@ -19,6 +19,11 @@ _LIB_NAME = "libfa.so"
 
 FA_OK = 0
 FA_ERR_DEVICE_TIMEOUT = 6
+FA_ERR_LAYOUT = 9
+
+# block of the block-sparse layout: query rows x keys (FA_BLOCK_Q, FA_BLOCK_K)
+BLOCK_Q = 256
+BLOCK_K = 128
 
 
 class FAError(RuntimeError):
@@ -70,6 +75,9 @@ def _load():
     lib.fa_bwd.restype = c_int
     lib.fa_bwd_workspace_bytes.argtypes = [c_int, c_int, c_int]
     lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.fa_fwd_block_sparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int,
+                                        c_float, c_int, vp]
+    lib.fa_fwd_block_sparse.restype = c_int
     lib.fa_version.argtypes = []
     lib.fa_version.restype = ctypes.c_char_p
     _lib = lib
@@ -177,6 +185,56 @@ def fa_fwd_splitkv(q, k, v, o, lse=None, workspace=None, num_splits: int = 0,
                               workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                               B, H, N, d, float(scale), int(bool(causal)), int(num_splits),
                               _stream_handle(stream)))
+
+
+def block_layout_to_csr(layout, device=None):
+    """CSR lists (row_ptr, col_idx), int32 on ``device``, of a boolean block layout.
+
+    layout[r][c] set = query block r (rows BLOCK_Q*r ...) retains key block c
+    (keys BLOCK_K*c ...); shape [ceil(N / BLOCK_Q), ceil(N / BLOCK_K)].
+    Column indices come out ascending within each row, as fa_fwd_block_sparse
+    requires.
+    """
+    lay = torch.as_tensor(layout, dtype=torch.bool, device=device)
+    if lay.dim() != 2:
+        raise ValueError("layout must be 2-D [query blocks, key blocks]")
+    counts = lay.sum(dim=1, dtype=torch.int32)
+    row_ptr = torch.zeros(lay.shape[0] + 1, dtype=torch.int32, device=lay.device)
+    row_ptr[1:] = torch.cumsum(counts, 0)
+    col_idx = lay.nonzero()[:, 1].to(torch.int32).contiguous()
+    return row_ptr, col_idx
+
+
+def fa_fwd_block_sparse(q, k, v, o, row_ptr, col_idx, lse=None, scale: float | None = None,
+                        causal: bool = False, stream=None) -> None:
+    """Block-sparse forward: attention over the key blocks each query block retains.
+
+    row_ptr, col_idx: CUDA int32 CSR lists (see block_layout_to_csr), one
+    layout for every (b, h).  Other arguments as fa_fwd.
+    """
+    lib = _load()
+    _check_qkvo(q, k, v, o)
+    B, H, N, d = q.shape
+    n_qb = -(-N // BLOCK_Q)
+    for name, t in (("row_ptr", row_ptr), ("col_idx", col_idx)):
+        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous() or t.dim() != 1:
+            raise ValueError(f"{name} must be a contiguous 1-D CUDA int32 tensor")
+    if row_ptr.numel() != n_qb + 1:
+        raise ValueError(f"row_ptr must have ceil(N / {BLOCK_Q}) + 1 = {n_qb + 1} entries")
+    lse_ptr = None
+    if lse is not None:
+        if lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous():
+            raise ValueError("lse must be a contiguous CUDA float32 tensor")
+        if tuple(lse.shape) != (B, H, N):
+            raise ValueError(f"lse must be [B, H, N] = {(B, H, N)}")
+        lse_ptr = lse.data_ptr()
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    nnz = col_idx.numel()
+    _check(lib.fa_fwd_block_sparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_ptr,
+                                   row_ptr.data_ptr(), col_idx.data_ptr() if nnz else None, nnz,
+                                   B, H, N, d, float(scale), int(bool(causal)),
+                                   _stream_handle(stream)))
 
 
 def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace=None, scale: float | None = None,

@@ -113,3 +113,56 @@ def sample_rows(B: int, H: int, N: int, count: int, seed: int) -> torch.Tensor:
     h = (idx // N) % H
     i = idx % N
     return torch.stack([b, h, i], dim=1)
+
+
+def make_local_qkv(B: int, H: int, N: int, d: int, seed: int, length_scale: float = 64.0,
+                   peak: float = 10.0):
+    """Q, K, V (CPU bf16 [B, H, N, d]) whose scores fall off with distance.
+
+    Half of each head's width carries random Fourier features of the
+    position: F = d/4 frequencies w ~ N(0, 1/length_scale^2) per head, a
+    cosine and a sine of w*i each, the same features in Q and K.  Their dot
+    product is a^2 sum_f cos(w_f (i - j)), whose mean over the frequencies is
+    a^2 F exp(-(i-j)^2 / (2 length_scale^2)); a is set so that, with the
+    scale 1/sqrt(d), this positional score is ``peak`` at distance 0.  The
+    other half of Q and K, and all of V, is N(0, 1).  Attention then
+    concentrates near the diagonal, the case where a block-sparse layout
+    that keeps a band of key blocks can match exact attention.
+
+    Recipe: a CPU generator seeded with ``seed`` draws the frequencies
+    [B, H, F], then the Q content, K content and V (float32 randn, in that
+    order); the features are computed in float64; everything is rounded to
+    bfloat16 at the end.
+    """
+    if d % 4:
+        raise ValueError("d must be a multiple of 4")
+    F = d // 4
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    w = torch.randn((B, H, F), generator=g, dtype=torch.float64) / float(length_scale)
+    qc = torch.randn((B, H, N, d // 2), generator=g, dtype=torch.float32)
+    kc = torch.randn((B, H, N, d // 2), generator=g, dtype=torch.float32)
+    v = torch.randn((B, H, N, d), generator=g, dtype=torch.float32)
+    a = math.sqrt(peak * math.sqrt(d) / F)
+    ang = torch.arange(N, dtype=torch.float64)[None, None, :, None] * w[:, :, None, :]
+    feat = (a * torch.cat([torch.cos(ang), torch.sin(ang)], dim=-1)).to(torch.float32)
+    q = torch.cat([feat, qc], dim=-1)
+    k = torch.cat([feat, kc], dim=-1)
+    return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+
+
+def local_block_layout(N: int, window: int, causal: bool, block_q: int, block_k: int,
+                       sinks: int = 0):
+    """Band layout: bool [ceil(N/block_q), ceil(N/block_k)] as nested lists.
+
+    Query block r retains key block c when c's keys meet the rows of r widened
+    by ``window`` keys to the left (and, unless causal, to the right), or when
+    c < ``sinks`` (the first key blocks, kept for every query block).
+    """
+    nqb, nkb = -(-N // block_q), -(-N // block_k)
+    lay = []
+    for r in range(nqb):
+        lo = r * block_q - window
+        hi = min(N, (r + 1) * block_q) - 1 + (0 if causal else window)
+        lay.append([(c < sinks) or (c * block_k <= hi and (c + 1) * block_k - 1 >= lo)
+                    for c in range(nkb)])
+    return lay

@@ -42,7 +42,8 @@ typedef enum fa_status {
   FA_ERR_CUDA = 5,            /* a CUDA runtime/driver call or the launch failed  */
   FA_ERR_DEVICE_TIMEOUT = 6,  /* a kernel gave up on a bounded wait               */
   FA_ERR_ALIAS = 7,           /* O, LSE or a workspace overlaps another argument  */
-  FA_ERR_WORKSPACE = 8        /* the workspace is smaller than required           */
+  FA_ERR_WORKSPACE = 8,       /* the workspace is smaller than required           */
+  FA_ERR_LAYOUT = 9           /* a block-sparse list was out of range or order    */
 } fa_status;
 
 /*
@@ -173,6 +174,45 @@ fa_status fa_fwd_splitkv_noalloc(const void* Q, const void* K, const void* V, vo
                                  int B, int H, int N, int d, float scale, int causal, int num_splits,
                                  void* stream);
 
+/* Block of the block-sparse layout: query rows x keys. */
+#define FA_BLOCK_Q 256
+#define FA_BLOCK_K 128
+
+/*
+ * fa_fwd_block_sparse -- attention over the key blocks a block layout
+ * retains: query i sees key j only if j's key block is in the list of i's
+ * query block (and j <= i when causal != 0).  The pages call sparsity a
+ * separate design dimension, choosing which query-key interactions are kept
+ * (liminalml.com "FlashAttention", "Is it sparse attention?"), and suggest
+ * comparing exact and block-sparse attention at matched output error
+ * (interactiveml.org "FlashAttention saves the matrix, not the quadratic
+ * work", the suggested experiments).  Over the retained keys the result is
+ * the exact softmax, computed as in fa_fwd; with every block retained it is
+ * fa_fwd's result, bit for bit.
+ *
+ *   Q, K, V, O, LSE, B, H, N, d, scale, causal, stream: as in fa_fwd.
+ *   block_row_ptr  device, int32 [ceil(N / FA_BLOCK_Q) + 1], read: query
+ *                  block r (rows FA_BLOCK_Q*r ...) retains the key blocks
+ *                  block_col_idx[block_row_ptr[r] .. block_row_ptr[r+1]-1].
+ *   block_col_idx  device, int32 [nnz], read: key block numbers (keys
+ *                  FA_BLOCK_K*c ...), strictly ascending within each query
+ *                  block, each in [0, ceil(N / FA_BLOCK_K)).  May be NULL when
+ *                  nnz == 0.
+ *   nnz            entries of block_col_idx (>= 0).
+ * One layout serves every (b, h).  A query with no retained key gets O = 0
+ * and LSE = -inf.  Key blocks past a causal block's last row are skipped.
+ *
+ * Errors: as fa_fwd, plus FA_ERR_NULL (no block_row_ptr, or no block_col_idx
+ * with nnz > 0), FA_ERR_SHAPE (nnz < 0), FA_ERR_ALIGN (a list not 4-byte
+ * aligned), FA_ERR_ALIAS (O or LSE overlaps a list).  The lists live on the
+ * device and are checked there: an entry out of range or out of order is
+ * masked out (nothing outside the tensors is read), the outputs are then
+ * undefined, and fa_get_device_status() reports FA_ERR_LAYOUT.
+ */
+fa_status fa_fwd_block_sparse(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                              const int* block_row_ptr, const int* block_col_idx, int nnz, int B,
+                              int H, int N, int d, float scale, int causal, void* stream);
+
 /*
  * fa_softmax_rows -- the softmax step of standard (materialising) attention,
  * kept as a comparator: standard attention writes the N x N scores to
@@ -200,15 +240,17 @@ const char* fa_status_string(fa_status status);
  * device status words (forward and backward kernels) of the current device.
  * Returns FA_ERR_DEVICE_TIMEOUT
  * if any kernel launched by this library gave up on a bounded wait since the
- * last call (its outputs are then undefined), FA_ERR_CUDA if the
- * synchronisation failed, FA_OK otherwise.
+ * last call (its outputs are then undefined), FA_ERR_LAYOUT if a
+ * block-sparse call met a malformed list (and no wait gave up), FA_ERR_CUDA
+ * if the synchronisation failed, FA_OK otherwise.
  */
 fa_status fa_get_device_status(void* stream);
 
 /*
  * fa_get_device_status_word -- as fa_get_device_status, and also stores the
- * raw status word in *word (0 = no failure; bit 0 = a wait gave up; bit 8+k =
- * the wait at site k gave up, for diagnosis).  word may be NULL.
+ * raw status word in *word (0 = no failure; bit 0 = a wait gave up; bit 1 = a
+ * malformed block-sparse list; bit 8+k = the wait at site k gave up, for
+ * diagnosis).  word may be NULL.
  */
 fa_status fa_get_device_status_word(void* stream, unsigned int* word);
 

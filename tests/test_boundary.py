@@ -17,6 +17,7 @@ LIB = os.path.join(ROOT, "exact_softmax_attention_02_b200", "libfa.so")
 
 FA_OK, FA_ERR_NULL, FA_ERR_SHAPE, FA_ERR_UNSUPPORTED, FA_ERR_ALIGN = 0, 1, 2, 3, 4
 FA_ERR_CUDA, FA_ERR_DEVICE_TIMEOUT, FA_ERR_ALIAS, FA_ERR_WORKSPACE = 5, 6, 7, 8
+FA_ERR_LAYOUT = 9
 
 
 @pytest.fixture(scope="module")
@@ -53,7 +54,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(9):
+    for code in range(10):
         s = lib.fa_status_string(code).decode()
         assert s.startswith("FA_")
     assert lib.fa_status_string(99).decode() == "unknown fa_status"
@@ -182,3 +183,25 @@ def test_bwd_argument_checks(lib):
     a = list(base)
     a[7] = base[7] + 8
     assert bwd(a) == FA_ERR_ALIGN
+
+
+def test_block_sparse_argument_checks(lib):
+    vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.fa_fwd_block_sparse.argtypes = [vp] * 7 + [ci] * 5 + [cf, ci, vp]
+    lib.fa_fwd_block_sparse.restype = ci
+    rp, ci_ = A + 320 * MB, A + 321 * MB
+
+    def bs(q=A, o=A + 192 * MB, lse=A + 256 * MB, row_ptr=rp, col_idx=ci_, nnz=4, N=1024, d=64):
+        return lib.fa_fwd_block_sparse(q, A + 64 * MB, A + 128 * MB, o, lse, row_ptr, col_idx, nnz,
+                                       1, 1, N, d, 0.125, 0, None)
+
+    assert bs(q=None) == FA_ERR_NULL
+    assert bs(row_ptr=None) == FA_ERR_NULL
+    assert bs(col_idx=None) == FA_ERR_NULL
+    assert bs(nnz=-1) == FA_ERR_SHAPE
+    assert bs(row_ptr=rp + 2) == FA_ERR_ALIGN
+    assert bs(col_idx=ci_ + 1) == FA_ERR_ALIGN
+    assert bs(d=96) == FA_ERR_UNSUPPORTED
+    assert bs(row_ptr=A + 192 * MB + 64) == FA_ERR_ALIAS  # list inside O
+    assert bs(col_idx=A + 256 * MB) == FA_ERR_ALIAS  # list inside LSE
+    assert lib.fa_status_string(FA_ERR_LAYOUT).decode().startswith("FA_ERR_LAYOUT")
