@@ -662,6 +662,56 @@ def run_sparse_experiment(args, w):
     return 0
 
 
+def run_tile_experiment(args, w):
+    """Wall-clock time of the fused forward against tile size and head width.
+
+    Key tiles of 64 and 128 (the query tile is the tensor core's 128 rows),
+    head widths 64 and 128, sequence lengths 1K to 64K with the token count
+    B*H*N fixed at 2^19 (so every point holds the same inputs), both masks.
+    One JSON line per point (CUDA-event time per launch, TFLOP/s), then one
+    line per (d, N, mask) naming the faster tile.  Inputs are N(0, 1), seeded.
+    """
+    import torch
+
+    from exact_softmax_attention_02_b200 import fa
+    from exact_softmax_attention_02_b200.inputs import make_qkv
+
+    if not torch.cuda.is_available():
+        raise SystemExit("the experiment needs a CUDA device")
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    steps, warmup = max(3, min(args.steps, 20)), args.warmup
+    tokens = 1 << 19
+    peak, peak_src = tensor_peak()
+    for d in (64, 128):
+        for N in (1024, 4096, 16384, 65536):
+            H = tokens // N
+            q_h, k_h, v_h = make_qkv(1, H, N, d, seed=N + d)
+            q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
+            o = torch.empty_like(q)
+            lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+            for causal in (False, True):
+                flops = 4.0 * H * N * N * d / (2 if causal else 1)
+                best = None
+                for key_tile in (64, 128):
+                    ms = time_launches(lambda: fa.fa_fwd_key_tile(q, k, v, o, lse, key_tile=key_tile,
+                                                                  causal=causal, stream=stream),
+                                       steps, warmup, stream)
+                    if fa.device_status(stream) != 0:
+                        raise RuntimeError("kernel reported a device failure")
+                    tf = flops / ms / 1e9
+                    pt = {"experiment": "tile_sweep", "B": 1, "H": H, "N": N, "d": d, "causal": causal,
+                          "query_tile": 128, "key_tile": key_tile, "ms": ms, "tflops": tf,
+                          "pct_of_peak": 100.0 * tf / peak, "peak_source": peak_src}
+                    print(json.dumps(pt), flush=True)
+                    if best is None or ms < best[1]:
+                        best = (key_tile, ms)
+                print(json.dumps({"experiment": "tile_sweep", "summary": True, "N": N, "d": d,
+                                  "causal": causal, "best_key_tile": best[0]}), flush=True)
+            del q, k, v, o, lse
+    return 0
+
+
 def main(argv=None):
     from exact_softmax_attention_02_b200.inputs import WORKLOADS
 
@@ -676,9 +726,10 @@ def main(argv=None):
                          "standard: the materialising comparator (GEMM, softmax, GEMM); "
                          "backward: fa_bwd (dQ, dK, dV)")
     ap.add_argument("--splits", type=int, default=0, help="splitkv: key ranges (0 = default)")
-    ap.add_argument("--experiment", default=None, choices=["sparse"],
-                    help="sparse: exact vs block-sparse bands at matched output error (1 GPU, "
-                         "JSON lines; not a bench line)")
+    ap.add_argument("--experiment", default=None, choices=["sparse", "tiles"],
+                    help="sparse: exact vs block-sparse bands at matched output error; tiles: "
+                         "time against key-tile width and head width (1 GPU, JSON lines; not a "
+                         "bench line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-step-seconds", type=float, default=8.0,
                     help="reference arm: target oracle seconds per step (bounded sample)")
@@ -699,6 +750,8 @@ def main(argv=None):
         return run_reference(args, w)
     if args.experiment == "sparse":
         return run_sparse_experiment(args, w)
+    if args.experiment == "tiles":
+        return run_tile_experiment(args, w)
     return run_ours(args, w)
 
 

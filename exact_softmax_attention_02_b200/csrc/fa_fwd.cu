@@ -61,7 +61,7 @@ cudaError_t read_and_clear_status(uint32_t* v);  // fa_bwd.cu
 }
 
 constexpr int kBM = 128;       // query rows per tile
-constexpr int kBN = 128;       // keys per tile
+constexpr int kBN = 128;       // keys per tile (default; 64 is built for the tile-size sweep)
 constexpr int kQTiles = 2;     // query tiles per CTA
 static_assert(FA_BLOCK_Q == kQTiles * kBM && FA_BLOCK_K == kBN,
               "a block-sparse block is one CTA's query rows by one key tile");
@@ -133,15 +133,18 @@ __device__ unsigned long long* g_trace;  // [kTraceCtas][4 roles][kTraceIters][8
   } while (0)
 #endif
 
-template <int D, bool PAIR>
+template <int D, bool PAIR, int BN = kBN>
 struct Cfg {
+  static_assert(BN == 128 || (BN == 64 && !PAIR), "key tiles of 128, or 64 on one CTA");
   static constexpr int kChunks = D / 64;
   static constexpr int kQBytes = kBM * D * 2;  // one query tile (reused as O staging)
   // one ring stage: a whole K or V tile, or (PAIR) this CTA's half of one
-  static constexpr int kStageBytes = PAIR ? kBM * D : kBM * D * 2;
-  static constexpr int kKRows = PAIR ? kBN / 2 : kBN;  // key rows of a K stage
-  static constexpr int kKChunkBytes = kKRows * 128;    // one 64-wide d chunk of a K stage
-  static constexpr int kStages = (PAIR || D == 64) ? 8 : 4;
+  static constexpr int kStageBytes = PAIR ? BN * D : BN * D * 2;
+  static constexpr int kKRows = PAIR ? BN / 2 : BN;  // key rows of a K stage
+  static constexpr int kKChunkBytes = kKRows * 128;  // one 64-wide d chunk of a K stage
+  static constexpr int kVChunkBytes = BN * 128;      // one 64-wide d chunk of a V stage
+  // the same ring bytes whatever the tile: more stages for smaller tiles
+  static constexpr int kStages = ((PAIR || D == 64) ? 8 : 4) * (128 / BN);
   static constexpr int kRowsPerTile = PAIR ? 2 * kBM : kBM;  // rows of one (pair) MMA tile
   static constexpr int kNumBars = 2 + 2 + 3 * kStages + 2 + 4 + 2 + 1 + 1;
   static constexpr int kSmemTiles = kQTiles * kQBytes + kStages * kStageBytes;
@@ -158,14 +161,16 @@ struct Cfg {
 // B and loads half of every K/V tile.  Each CTA's TMA signals a local barrier;
 // a forwarding warp then arrives on the even CTA's barrier, so that both CTAs
 // can drain their own copies exactly if they have to unwind.
-template <int D, bool CAUSAL, bool PAIR, bool SPLIT, bool SPARSE>
+template <int D, bool CAUSAL, bool PAIR, bool SPLIT, bool SPARSE, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const FwdParams p) {
-  using C = Cfg<D, PAIR>;
+  using C = Cfg<D, PAIR, BN>;
   constexpr int S = C::kStages;
   constexpr int QB = C::kQBytes;
+  static_assert(BN == BN || !(SPLIT || SPARSE), "split-KV and block-sparse use 128-key tiles");
+  static_assert(BN == 128 || kPHalves == 1, "P is published in halves only with 128-key tiles");
   constexpr int SB = C::kStageBytes;
   static_assert(!PAIR || D == 128, "the pair kernel splits d = 128 into two 64-wide halves");
   static_assert(!(PAIR && SPLIT), "split-KV uses the single-CTA shape");
@@ -217,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int j_last[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t)
-    j_last[t] = CAUSAL ? min(q0 + (t + 1) * C::kRowsPerTile - 1, p.N - 1) / kBN : p.n_kv - 1;
+    j_last[t] = CAUSAL ? min(q0 + (t + 1) * C::kRowsPerTile - 1, p.N - 1) / BN : p.n_kv - 1;
   // key tiles [kv_lo, kv_end) of this CTA (all of them unless split), visited
   // from kv_end-1 down to kv_lo
   const int kv_lo = SPLIT ? split * p.kv_per_split : 0;
@@ -320,12 +325,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (kv == 0) {
             for (int c = 0; c < C::kChunks; ++c)
               tma_load_3d(st + c * C::kKChunkBytes, &tmK, &kv_land[s], c * 64,
-                          j * kBN + static_cast<int>(rank) * C::kKRows, bh);
+                          j * BN + static_cast<int>(rank) * C::kKRows, bh);
           } else if (PAIR) {
-            tma_load_3d(st, &tmV, &kv_land[s], static_cast<int>(rank) * 64, j * kBN, bh);
+            tma_load_3d(st, &tmV, &kv_land[s], static_cast<int>(rank) * 64, j * BN, bh);
           } else {
             for (int c = 0; c < C::kChunks; ++c)
-              tma_load_3d(st + c * kChunkBytes, &tmV, &kv_land[s], c * 64, j * kBN, bh);
+              tma_load_3d(st + c * C::kVChunkBytes, &tmV, &kv_land[s], c * 64, j * BN, bh);
           }
           ++i;
           if (it == 0 && kv == 0) {
@@ -367,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && rank == 0 && n_iter > 0) {
       constexpr uint32_t kM = PAIR ? 2 * kBM : kBM;
-      constexpr uint32_t idS = idesc_bf16_f32(kM, kBN, false);
+      constexpr uint32_t idS = idesc_bf16_f32(kM, BN, false);
       constexpr uint32_t idO = idesc_bf16_f32(kM, D, true);
       const uint32_t sq = smem_addr(sQ);
       const uint32_t skv = smem_addr(sKV);
@@ -380,22 +385,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd =
               sw128_desc(skv + s * SB + (kk >> 2) * C::kKChunkBytes + (kk & 3) * 32, 16, 1024);
           if (PAIR)
-            mma_ss_pair(tmem + t * kBN, ad, bd, idS, kk > 0 ? 1u : 0u);
+            mma_ss_pair(tmem + t * BN, ad, bd, idS, kk > 0 ? 1u : 0u);
           else
-            mma_ss(tmem + t * kBN, ad, bd, idS, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + t * BN, ad, bd, idS, kk > 0 ? 1u : 0u);
         }
       };
       // O_t (+)= P_t V: A = P_t in TMEM (8 columns per 16 keys), B = V stage
       // stored d-contiguous (MN-major): 16 keys = 2 KB apart, d halves 16 KB apart.
       auto issue_pv = [&](int t, int s, bool accumulate, int half) {
 #pragma unroll
-        for (int kk = half * (kBN / 32); kk < (half + 1) * (kBN / 32); ++kk) {
-          const uint64_t bd = sw128_desc(skv + s * SB + kk * 2048, kChunkBytes, 1024);
+        for (int kk = half * (BN / 32); kk < (half + 1) * (BN / 32); ++kk) {
+          const uint64_t bd = sw128_desc(skv + s * SB + kk * 2048, C::kVChunkBytes, 1024);
           const uint32_t acc = (accumulate || kk > 0) ? 1u : 0u;
           if (PAIR)
-            mma_ts_pair(tmem + C::kColO + t * D, tmem + t * kBN + kk * 8, bd, idO, acc);
+            mma_ts_pair(tmem + C::kColO + t * D, tmem + t * BN + kk * 8, bd, idO, acc);
           else
-            mma_ts(tmem + C::kColO + t * D, tmem + t * kBN + kk * 8, bd, idO, acc);
+            mma_ts(tmem + C::kColO + t * D, tmem + t * BN + kk * 8, bd, idO, acc);
         }
       };
       auto commit = [&](uint64_t* bar) {
@@ -475,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row0 = tile_row0(t);
     const int row = row0 + r;                   // query index in the head
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_base + t * kBN;
+    const uint32_t tS = tmem + lane_base + t * BN;
     const uint32_t tO = tmem + lane_base + C::kColO + t * D;
     const float sl2 = p.scale_log2;
     // last key this row may see
@@ -519,37 +524,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool tr = lane == 0 && (warp & 3) == 0;
       if (tr) FA_TRACE_MARK(1 + t, it, 0);
       tc_fence_after();
-      uint32_t sr[4][32];
+      constexpr int kQ32 = BN / 32;  // 32-key groups of a tile
+      uint32_t sr[kQ32][32];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, sr[q]);
+      for (int q = 0; q < kQ32; ++q) tmem_ld32(tS + q * 32, sr[q]);
       tmem_wait_ld();
       if (tr) FA_TRACE_MARK(1 + t, it, 1);
 
-      const int kbase = j * kBN;
-      const bool masked = bad || (kbase + kBN > p.N) || (CAUSAL && kbase + kBN - 1 > row0);
+      const int kbase = j * BN;
+      const bool masked = bad || (kbase + BN > p.N) || (CAUSAL && kbase + BN - 1 > row0);
       if (masked) {
         const int lim = bad ? -1 : key_limit;
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < kQ32; ++q)
 #pragma unroll
           for (int c = 0; c < 32; ++c)
             if (kbase + q * 32 + c > lim) sr[q][c] = __float_as_uint(-INFINITY);
       }
-      // row maximum of the raw scores (scale > 0 keeps the argmax): eight
+      // row maximum of the raw scores (scale > 0 keeps the argmax): BN/16
       // independent chains of three-input maxima
-      float mx[8];
+      constexpr int kChains = BN / 16;
+      float mx[kChains];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(sr[k >> 1][(k & 1) * 16]);
+      for (int k = 0; k < kChains; ++k) mx[k] = __uint_as_float(sr[k >> 1][(k & 1) * 16]);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
+      for (int k = 0; k < kChains; ++k) {
         const uint32_t* v = &sr[k >> 1][(k & 1) * 16];
 #pragma unroll
         for (int c = 1; c < 15; c += 2)
           mx[k] = fmax3(mx[k], __uint_as_float(v[c]), __uint_as_float(v[c + 1]));
         mx[k] = fmaxf(mx[k], __uint_as_float(v[15]));
       }
-      const float m_tile =
-          fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * sl2;
+      float m_all;
+      if constexpr (kChains == 8)
+        m_all = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+      else
+        m_all = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]);
+      const float m_tile = m_all * sl2;
       if (tr) FA_TRACE_MARK(1 + t, it, 2);
       // raise the reference maximum only when this tile exceeds it by > 2^8
       const bool raise = m_tile > m_ref + kRescaleThreshold;
@@ -563,14 +574,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
       const float2 sl2v = make_float2(sl2, sl2);
       const float2 nm2 = make_float2(neg_m, neg_m);
-      float2 ps2[4];
+      float2 ps2[kQ32];
       // p = 2^(s * scale * log2 e - m) (the last kEmuPer32 columns of every
       // 32 on the FMA pipe, the rest on MUFU), written as bf16 pairs over the
-      // first 64 columns of S_t in two halves of 64 keys, published on
+      // first BN/2 columns of S_t in halves of 64 keys, published on
       // p_half[2t] (whole tile) or, with kPHalves == 2, each half on its own
       // barrier p_half[2t+h] as soon as it is in TMEM.
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      for (int h = 0; h < BN / 64; ++h) {
+        constexpr int kLastH = BN / 64 - 1;
         uint32_t pk[32];
 #pragma unroll
         for (int qq = 0; qq < 2; ++qq) {
@@ -593,8 +605,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st32(tS + h * 32, pk);
         // whole-P: the rescale waits until the scores have left the registers
-        if (kPHalves == 1 && h == 1 && rescale_o) rescale_o_rows(tO, alpha);
-        if (kPHalves == 2 || h == 1) {
+        if (kPHalves == 1 && h == kLastH && rescale_o) rescale_o_rows(tO, alpha);
+        if (kPHalves == 2 || h == kLastH) {
           tmem_wait_st();
           tc_fence_before();
           uint64_t* pbar = &p_half[2 * t + ((kPHalves == 2 && h == 1) ? 1 : 0)];
@@ -609,7 +621,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (tr && h == 0) FA_TRACE_MARK(1 + t, it, 3);
       }
-      const float2 psum = fadd2(fadd2(ps2[0], ps2[1]), fadd2(ps2[2], ps2[3]));
+      float2 psum;
+      if constexpr (kQ32 == 4)
+        psum = fadd2(fadd2(ps2[0], ps2[1]), fadd2(ps2[2], ps2[3]));
+      else
+        psum = fadd2(ps2[0], ps2[1]);
       l_sum = l_sum * alpha + (psum.x + psum.y);
       if (tr) FA_TRACE_MARK(1 + t, it, 4);
     }
@@ -770,7 +786,7 @@ using host::overlaps;
 struct DeviceInfo {
   bool checked = false;
   bool sm100 = false;
-  bool attr_set[32] = {};
+  bool attr_set[64] = {};
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_devices[kMaxDevices];
@@ -787,14 +803,15 @@ template <int D>
 constexpr bool kUsePair = false;
 #endif
 
-template <int D, bool CAUSAL, bool SPLIT, bool SPARSE = false>
+template <int D, bool CAUSAL, bool SPLIT, bool SPARSE = false, int BN = kBN>
 fa_status launch(const void* Q, const void* K, const void* V, void* O, FwdParams prm, int N, int BH,
                  cudaStream_t stream, DeviceInfo& dev) {
-  constexpr bool PAIR = kUsePair<D> && !SPLIT && !SPARSE;
-  using C = Cfg<D, PAIR>;
+  constexpr bool PAIR = kUsePair<D> && !SPLIT && !SPARSE && BN == kBN;
+  using C = Cfg<D, PAIR, BN>;
+  prm.n_kv = (N + BN - 1) / BN;
   CUtensorMap mq, mk, mv, mo;
   if (!make_map(&mq, Q, D, N, BH, kBM) || !make_map(&mk, K, D, N, BH, C::kKRows) ||
-      !make_map(&mv, V, D, N, BH, kBM) || !make_map(&mo, O, D, N, BH, kBM)) {
+      !make_map(&mv, V, D, N, BH, BN) || !make_map(&mo, O, D, N, BH, kBM)) {
     snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed");
     return FA_ERR_CUDA;
   }
@@ -803,9 +820,9 @@ fa_status launch(const void* Q, const void* K, const void* V, void* O, FwdParams
   const long long units = static_cast<long long>(BH) * prm.n_qblk;
   const long long grid = units * (SPLIT ? prm.num_splits : (PAIR ? 2 : 1));
   if (grid > 0x7fffffffll) return FA_ERR_SHAPE;
-  constexpr int slot =
-      (SPARSE ? 16 : 0) + (D == 128 ? 8 : 0) + (CAUSAL ? 4 : 0) + (PAIR ? 2 : 0) + (SPLIT ? 1 : 0);
-  auto kern = fa_fwd_kernel<D, CAUSAL, PAIR, SPLIT, SPARSE>;
+  constexpr int slot = (BN == 64 ? 32 : 0) + (SPARSE ? 16 : 0) + (D == 128 ? 8 : 0) + (CAUSAL ? 4 : 0) +
+                       (PAIR ? 2 : 0) + (SPLIT ? 1 : 0);
+  auto kern = fa_fwd_kernel<D, CAUSAL, PAIR, SPLIT, SPARSE, BN>;
   if (!dev.attr_set[slot]) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -994,6 +1011,27 @@ fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
                   : launch<128, false, false>(Q, K, V, O, prm, N, bh, st, *dev);
   return causal ? launch<64, true, false>(Q, K, V, O, prm, N, bh, st, *dev)
                 : launch<64, false, false>(Q, K, V, O, prm, N, bh, st, *dev);
+}
+
+fa_status fa_fwd_key_tile(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                          int H, int N, int d, float scale, int causal, int key_tile, void* stream) {
+  using namespace fa;
+  if (key_tile == 0 || key_tile == kBN) return fa_fwd(Q, K, V, O, LSE, B, H, N, d, scale, causal, stream);
+  FwdParams prm;
+  DeviceInfo* dev = nullptr;
+  fa_status st0 = check_args(Q, K, V, O, LSE, B, H, N, d, scale);
+  if (st0 != FA_OK) return st0;
+  if (key_tile != 64) return FA_ERR_UNSUPPORTED;
+  st0 = prepare(LSE, B, H, N, d, scale, &prm, &dev);
+  if (st0 != FA_OK) return st0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int bh = prm.BH;
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  if (d == 128)
+    return causal ? launch<128, true, false, false, 64>(Q, K, V, O, prm, N, bh, st, *dev)
+                  : launch<128, false, false, false, 64>(Q, K, V, O, prm, N, bh, st, *dev);
+  return causal ? launch<64, true, false, false, 64>(Q, K, V, O, prm, N, bh, st, *dev)
+                : launch<64, false, false, false, 64>(Q, K, V, O, prm, N, bh, st, *dev);
 }
 
 int fa_fwd_splitkv_default_splits(int B, int H, int N, int d, int causal) {

@@ -78,6 +78,9 @@ def _load():
     lib.fa_fwd_block_sparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int,
                                         c_float, c_int, vp]
     lib.fa_fwd_block_sparse.restype = c_int
+    lib.fa_fwd_key_tile.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_float, c_int, c_int,
+                                    vp]
+    lib.fa_fwd_key_tile.restype = c_int
     lib.fa_version.argtypes = []
     lib.fa_version.restype = ctypes.c_char_p
     _lib = lib
@@ -133,6 +136,26 @@ def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
         scale = 1.0 / math.sqrt(d)
     _check(lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_ptr,
                       B, H, N, d, float(scale), int(bool(causal)), _stream_handle(stream)))
+
+
+def fa_fwd_key_tile(q, k, v, o, lse=None, key_tile: int = 128, scale: float | None = None,
+                    causal: bool = False, stream=None) -> None:
+    """fa_fwd on 128 x ``key_tile`` score tiles (64 or 128), for the tile-size sweep."""
+    lib = _load()
+    _check_qkvo(q, k, v, o)
+    B, H, N, d = q.shape
+    lse_ptr = None
+    if lse is not None:
+        if lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous():
+            raise ValueError("lse must be a contiguous CUDA float32 tensor")
+        if tuple(lse.shape) != (B, H, N):
+            raise ValueError(f"lse must be [B, H, N] = {(B, H, N)}")
+        lse_ptr = lse.data_ptr()
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    _check(lib.fa_fwd_key_tile(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_ptr,
+                               B, H, N, d, float(scale), int(bool(causal)), int(key_tile),
+                               _stream_handle(stream)))
 
 
 def _check_qkvo(q, k, v, o):

@@ -174,6 +174,20 @@ fa_status fa_fwd_splitkv_noalloc(const void* Q, const void* K, const void* V, vo
                                  int B, int H, int N, int d, float scale, int causal, int num_splits,
                                  void* stream);
 
+/*
+ * fa_fwd_key_tile -- fa_fwd with a chosen key-tile width, for measuring how
+ * wall-clock time depends on the tile size (interactiveml.org
+ * "FlashAttention saves the matrix, not the quadratic work", the suggested
+ * experiments: vary tile size and head width).  key_tile = 128 (or 0) is
+ * fa_fwd itself; key_tile = 64 runs the same kernel on 128 x 64 score tiles
+ * (twice the key tiles, each half as wide, with a ring of twice as many
+ * stages).  The query tile stays 128 rows: the tensor core's M.  Results
+ * agree with fa_fwd to rounding.  Arguments and errors as fa_fwd, plus
+ * FA_ERR_UNSUPPORTED for any other key_tile.
+ */
+fa_status fa_fwd_key_tile(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                          int H, int N, int d, float scale, int causal, int key_tile, void* stream);
+
 /* Block of the block-sparse layout: query rows x keys. */
 #define FA_BLOCK_Q 256
 #define FA_BLOCK_K 128

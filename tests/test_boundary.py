@@ -205,3 +205,19 @@ def test_block_sparse_argument_checks(lib):
     assert bs(row_ptr=A + 192 * MB + 64) == FA_ERR_ALIAS  # list inside O
     assert bs(col_idx=A + 256 * MB) == FA_ERR_ALIAS  # list inside LSE
     assert lib.fa_status_string(FA_ERR_LAYOUT).decode().startswith("FA_ERR_LAYOUT")
+
+
+def test_key_tile_argument_checks(lib):
+    vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.fa_fwd_key_tile.argtypes = [vp] * 5 + [ci] * 4 + [cf, ci, ci, vp]
+    lib.fa_fwd_key_tile.restype = ci
+
+    def kt(key_tile, q=A, d=64):
+        return lib.fa_fwd_key_tile(q, A + 64 * MB, A + 128 * MB, A + 192 * MB, A + 256 * MB,
+                                   1, 1, 1024, d, 0.125, 0, key_tile, None)
+
+    assert kt(96) == FA_ERR_UNSUPPORTED
+    assert kt(256) == FA_ERR_UNSUPPORTED
+    assert kt(64, q=None) == FA_ERR_NULL
+    assert kt(64, d=32) == FA_ERR_UNSUPPORTED
+    assert kt(128, q=A + 8) == FA_ERR_ALIGN
