@@ -351,7 +351,8 @@ def run_ours(args, w):
         g = torch.Generator(device="cpu").manual_seed(w.seed + 100)
         do = torch.randn(q.shape, generator=g).to(torch.bfloat16).to(dev)
         bwd = dict(do=do, dq=torch.empty_like(q), dk=torch.empty_like(q), dv=torch.empty_like(q),
-                   ws=torch.empty(max(16, w.B * w.H * w.N * 4), dtype=torch.uint8, device=dev))
+                   ws=torch.empty(max(16, fa.bwd_workspace_bytes(w.B, w.H, w.N)), dtype=torch.uint8,
+                                  device=dev))
         launches_per_step = 3  # D = rowsum(dO*O), dK/dV, dQ
     if args.path == "splitkv":
         splits = args.splits if args.splits > 0 else fa.splitkv_default_splits(w.B, w.H, w.N, w.d, w.causal)

@@ -10,7 +10,8 @@
 //   dQ = scale dS K,  dK = scale dS^T Q.
 //
 // Three kernels:
-//   bwd_rowdot   D = rowsum(dO * O), one warp per row (HBM-bound).
+//   bwd_rowdot   D = rowsum(dO * O) and LSE * log2(e), one warp per row,
+//                into a workspace padded to whole 128-row tiles (HBM-bound).
 //   bwd_dkdv     one CTA per 128-key tile: S^T = K Q^T and dP^T = V dO^T into
 //                TMEM, P^T and dS^T formed in place (bf16), then
 //                dV += P^T dO and dK += dS^T Q accumulate in TMEM over the
@@ -19,7 +20,14 @@
 //                place, dQ += dS K over the key tiles.
 // CTA layout of the two tiled kernels (384 threads): warp 0 TMA producer,
 // warp 1 TMEM owner and MMA issuer, warps 4-11 elementwise step and epilogue
-// (two threads per TMEM lane, i.e. per row of the tile, 64 columns each).
+// (two threads per TMEM lane, i.e. per row).  The elementwise threads work
+// through each tile a quarter (32 columns) at a time and release every
+// quarter to the MMA issuer on its own barrier, so that the accumulating
+// products of one quarter overlap the elementwise step of the next.  The
+// MMAs are all N = 128 (S, dP) or N = d (accumulators): issuing a
+// tcgen05.mma takes its thread about as long as an M = 128, N = 128, K = 16
+// product runs, so narrower products would leave the tensor core waiting on
+// issue.
 // Every wait is bounded as in the forward kernel.
 
 #include <cuda.h>
@@ -38,37 +46,58 @@
 namespace fa {
 namespace bwd {
 
-constexpr int kTile = 128;   // rows of a query tile, keys of a key tile
+constexpr int kTile = 128;  // query rows and keys per tile
+constexpr int kQuarter = 32;  // columns released to the MMAs at a time
 constexpr int kThreads = 384;
-constexpr int kElemWarp0 = 4;
-constexpr int kElemThreads = 256;  // warps 4-11: two threads per row, 64 columns each
+constexpr int kElemWarp0 = 4;      // warps 4-11: two threads per row, 16 columns of each quarter each
+constexpr int kElemThreads = 256;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kChunkBytes = kTile * 64 * 2;  // one 64-wide, 128-row swizzled box
+constexpr int kChunkBytes = kTile * 64 * 2;  // one 64-wide, 128-row swizzled box: 16 KB
 
 enum : uint32_t { kSiteLoad = 0, kSiteStage = 1, kSiteS = 2, kSiteDs = 3, kSiteO = 4 };
 
 struct BwdParams {
-  const float* lse;  // [BH][N] natural-log LSE of the forward
-  const float* dd;   // [BH][N] D = rowsum(dO * O)
+  const float* lse2;  // [BH][n_pad] the forward's LSE times log2(e); +inf past N
+  const float* dd;    // [BH][n_pad] D = rowsum(dO * O); 0 past N
   int N;
+  int n_pad;          // N rounded up to a multiple of 128
   int BH;
-  int n_tiles;       // ceil(N / 128)
-  int group_heads;   // heads whose CTAs are scheduled together
-  float scale;       // multiplier of q.k
-  float scale_log2;  // scale * log2(e)
+  int n_tiles;        // n_pad / 128
+  int group_heads;    // heads whose CTAs are scheduled together
+  float scale;        // multiplier of q.k
+  float scale_log2;   // scale * log2(e)
   uint64_t timeout_ns;
 };
 
 __device__ uint32_t g_bwd_status;
 
-// TMEM column maps (both kernels): S or S^T at [0,128), dP or dP^T at
-// [128,256), accumulators from 256.  P / dS (bf16 pairs) overwrite their own
-// tile: the 32 values of columns 32c..32c+31 go, packed, to columns
-// 32c..32c+15, so each thread only overwrites what it has already read.
-constexpr uint32_t kColS = 0, kColDP = 128, kColAcc = 256;
+// Optional phase trace (build with -DFA_TRACE): SM clock stamps of the
+// producer, the MMA issuer and two elementwise threads, for the first CTAs
+// of each tiled kernel (k = 0: dK/dV, 1: dQ).
+#ifdef FA_TRACE
+constexpr int kTraceCtas = 16;
+constexpr int kTraceIters = 64;
+__device__ unsigned long long* g_bwd_trace;  // [2][kTraceCtas][4 roles][kTraceIters][8 events]
+#define BWD_TRACE(k, role, iter, ev)                                                                   \
+  do {                                                                                                 \
+    if (g_bwd_trace != nullptr && blockIdx.x < kTraceCtas && (iter) < kTraceIters)                     \
+      g_bwd_trace[(((static_cast<size_t>(k) * kTraceCtas + blockIdx.x) * 4 + (role)) * kTraceIters +   \
+                   (iter)) * 8 + (ev)] = clock64();                                                     \
+  } while (0)
+#else
+#define BWD_TRACE(k, role, iter, ev) \
+  do {                               \
+  } while (0)
+#endif
 
-// TMEM column of the packed bf16 operand for K-step kk (16 keys or queries)
-__device__ __forceinline__ uint32_t packed_col(int kk) { return (kk >> 1) * 32 + (kk & 1) * 8; }
+// TMEM columns (both tiled kernels): S (or S^T) at [0,128), dP (or dP^T) at
+// [128,256), accumulators from 256.  P and dS (bf16 pairs) overwrite their own
+// columns: the 16 values a thread forms in columns c..c+15 go, packed, to
+// columns c..c+7.
+constexpr uint32_t kColS = 0, kColDP = 128, kColAcc = 256;
+// TMEM column of the packed bf16 operand for K-step kk (16 queries or keys):
+// quarter kk / 2, half kk % 2
+__device__ __forceinline__ uint32_t packed_col(int kk) { return (kk >> 1) * 32 + (kk & 1) * 16; }
 
 // Work order shared by the tiled kernels: heads in groups, inside a group the
 // tiles with the most work first, cycling over the group's heads.
@@ -82,35 +111,64 @@ __device__ __forceinline__ void tile_of(const BwdParams& p, bool heavy_high, int
   *tile = heavy_high ? p.n_tiles - 1 - k : k;
 }
 
-// Elementwise step over 64 of the 128 columns (chunks c0, c0+1 of 32) of the
-// calling thread's row: p = 2^(s * scale log2e - lse2), masked to 0 where
-// `allowed` fails; ds = p * (dp - dsub).  P (optional) and dS are written as
-// bf16 pairs into the first half of each chunk's own columns.
-template <bool WRITE_P, typename ColLse, typename ColDsub, typename Allowed>
-__device__ __forceinline__ void p_ds_tile(uint32_t tS, uint32_t tDP, int c0, float sl2, ColLse col_lse2,
-                                          ColDsub col_dsub, Allowed allowed) {
+// Elementwise step on 16 columns c0..c0+15 of the calling thread's row, on
+// scores s and dp already in registers: p = 2^(s * scale log2e - lse2), 0
+// where `allowed` fails (MASK only); ds = p * (dp - D).  col(c, l4, d4) gives
+// lse2 and D of columns c..c+3.  P (optional) and dS are written back as 8
+// columns of bf16 pairs at c0.
+template <bool WRITE_P, bool MASK, typename Col, typename Allowed>
+__device__ __forceinline__ void p_ds_16(const uint32_t (&s)[16], const uint32_t (&dp)[16], uint32_t tS,
+                                        uint32_t tDP, int c0, float sl2, Col col, Allowed allowed) {
+  uint32_t pk[8], dk[8];
+  const float2 sl2v = make_float2(sl2, sl2);
 #pragma unroll
-  for (int cc = 0; cc < 2; ++cc) {
-    const int c = c0 + cc;
-    uint32_t s[32], dp[32];
-    tmem_ld32(tS + c * 32, s);
-    tmem_ld32(tDP + c * 32, dp);
-    tmem_wait_ld();
-    uint32_t pk[16], dk[16];
+  for (int e = 0; e < 16; e += 4) {
+    float4 l4, d4;
+    col(c0 + e, l4, d4);
 #pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-      const int col0 = c * 32 + e, col1 = col0 + 1;
-      float p0 = ex2_approx(fmaf(__uint_as_float(s[e]), sl2, -col_lse2(col0)));
-      float p1 = ex2_approx(fmaf(__uint_as_float(s[e + 1]), sl2, -col_lse2(col1)));
-      if (!allowed(col0)) p0 = 0.f;
-      if (!allowed(col1)) p1 = 0.f;
-      const float d0 = p0 * (__uint_as_float(dp[e]) - col_dsub(col0));
-      const float d1 = p1 * (__uint_as_float(dp[e + 1]) - col_dsub(col1));
-      pk[e >> 1] = pack_bf16x2(p0, p1);
-      dk[e >> 1] = pack_bf16x2(d0, d1);
+    for (int u = 0; u < 4; u += 2) {
+      const float2 sv = make_float2(__uint_as_float(s[e + u]), __uint_as_float(s[e + u + 1]));
+      const float2 lv = u == 0 ? make_float2(-l4.x, -l4.y) : make_float2(-l4.z, -l4.w);
+      const float2 dv = u == 0 ? make_float2(-d4.x, -d4.y) : make_float2(-d4.z, -d4.w);
+      const float2 x = ffma2(sv, sl2v, lv);
+      float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      if (MASK) {
+        if (!allowed(c0 + e + u)) pv.x = 0.f;
+        if (!allowed(c0 + e + u + 1)) pv.y = 0.f;
+      }
+      const float2 g = fadd2(make_float2(__uint_as_float(dp[e + u]), __uint_as_float(dp[e + u + 1])), dv);
+      const float2 dsv = fmul2(pv, g);
+      pk[(e + u) >> 1] = pack_bf16x2(pv.x, pv.y);
+      dk[(e + u) >> 1] = pack_bf16x2(dsv.x, dsv.y);
     }
-    if (WRITE_P) tmem_st16(tS + c * 32, pk);
-    tmem_st16(tDP + c * 32, dk);
+  }
+  if (WRITE_P) tmem_st8(tS + c0, pk);
+  tmem_st8(tDP + c0, dk);
+}
+
+// The calling thread's share of one tile: 16 columns of each quarter
+// (column h*16 of quarters 0..3), quarter by quarter.  The TMEM loads of the
+// next quarter are issued before the current one is computed; after its
+// stores have completed, each quarter is released on ready[q].
+template <bool WRITE_P, bool MASK, typename Col, typename Allowed>
+__device__ __forceinline__ void p_ds_tile(uint32_t tS, uint32_t tDP, int h, float sl2, Col col,
+                                          Allowed allowed, uint64_t* ready) {
+  uint32_t s[2][16], dp[2][16];
+  tmem_ld16(tS + h * 16, s[0]);
+  tmem_ld16(tDP + h * 16, dp[0]);
+  tmem_wait_ld_regs(s[0], dp[0]);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int c0 = q * kQuarter + h * 16;
+    if (q < 3) {
+      tmem_ld16(tS + c0 + kQuarter, s[(q + 1) & 1]);
+      tmem_ld16(tDP + c0 + kQuarter, dp[(q + 1) & 1]);
+    }
+    p_ds_16<WRITE_P, MASK>(s[q & 1], dp[q & 1], tS, tDP, c0, sl2, col, allowed);
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(&ready[q]);
+    if (q < 3) tmem_wait_ld_regs(s[(q + 1) & 1], dp[(q + 1) & 1]);
   }
 }
 
@@ -141,18 +199,29 @@ __device__ __forceinline__ void store_tile(uint32_t tAcc, float mul, uint8_t* st
 }
 
 // ---------------------------------------------------------------------------
-// D = rowsum(dO * O)
+// D = rowsum(dO * O) and LSE in log2 units, padded to n_pad rows per head
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256)
     bwd_rowdot_kernel(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __restrict__ dO,
-                      float* __restrict__ dd, long long rows) {
+                      const float* __restrict__ lse, float* __restrict__ lse2, float* __restrict__ dd,
+                      int N, int n_pad, long long rows_pad) {
   constexpr int kPer = D / 32;
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  const __nv_bfloat162* o = reinterpret_cast<const __nv_bfloat162*>(O + row * D + lane * kPer);
-  const __nv_bfloat162* g = reinterpret_cast<const __nv_bfloat162*>(dO + row * D + lane * kPer);
+  if (row >= rows_pad) return;
+  const long long bh = row / n_pad;
+  const int q = static_cast<int>(row - bh * n_pad);
+  if (q >= N) {  // padding: P = 0 there
+    if (lane == 0) {
+      lse2[row] = INFINITY;
+      dd[row] = 0.f;
+    }
+    return;
+  }
+  const long long src = bh * N + q;
+  const __nv_bfloat162* o = reinterpret_cast<const __nv_bfloat162*>(O + src * D + lane * kPer);
+  const __nv_bfloat162* g = reinterpret_cast<const __nv_bfloat162*>(dO + src * D + lane * kPer);
   float acc = 0.f;
 #pragma unroll
   for (int i = 0; i < kPer / 2; ++i) {
@@ -162,23 +231,33 @@ __global__ void __launch_bounds__(256)
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) dd[row] = acc;
+  if (lane == 0) {
+    dd[row] = acc;
+    lse2[row] = lse[src] * 1.4426950408889634f;
+  }
 }
 
 // ---------------------------------------------------------------------------
-// dK, dV: one CTA per key tile
+// dK, dV: one CTA per 128-key tile
 // ---------------------------------------------------------------------------
 template <int D>
 struct DkdvCfg {
   static constexpr int kChunks = D / 64;
   static constexpr int kTileBytes = kTile * D * 2;
-  static constexpr int kStages = D == 128 ? 2 : 3;      // each stage: Q_i and dO_i
+  static constexpr int kStages = D == 128 ? 2 : 4;  // each stage: Q_i and dO_i (+ LSE2_i, D_i)
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kSmemTiles = 2 * kTileBytes + kStages * kStageBytes;  // K, V, ring
-  static constexpr int kNumBars = 1 + 2 * kStages + 1 + 1 + 1 + 1;
-  static constexpr int kSmemBytes = kSmemTiles + 2 * 2 * kTile * 4 + kNumBars * 8 + 16 + 1024;
+  static constexpr int kLdBytes = kStages * 2 * kTile * 4;
+  static constexpr int kNumBars = 1 + 2 * kStages + 1 + 4 + 1 + 1;
+  static constexpr int kSmemBytes = kSmemTiles + kLdBytes + kNumBars * 8 + 16 + 1024;
 };
 
+// Per query tile i: S^T = K Q_i^T and dP^T = V dO_i^T (N = 128) into TMEM;
+// the elementwise threads then form P^T and dS^T a quarter (32 queries) at a
+// time and release each quarter on its own barrier, so that dV += P^T dO and
+// dK += dS^T Q run on one quarter while the next is being formed.  tcgen05
+// MMAs of one thread run in issue order, so the S^T of tile i+1 may be issued
+// right after the products that read tile i's P^T and dS^T.
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -193,16 +272,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sK = smem;
   uint8_t* sV = smem + TB;
-  uint8_t* sRing = smem + 2 * TB;  // stage s: Q at +0, dO at +TB
-  float* sLse = reinterpret_cast<float*>(smem + C::kSmemTiles);  // [2][128] log2 units
-  float* sD = sLse + 2 * kTile;                                   // [2][128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sD + 2 * kTile);
-  uint64_t* kv_full = bars;            // K_j, V_j landed
-  uint64_t* st_full = bars + 1;        // [S] Q_i, dO_i landed
-  uint64_t* st_empty = st_full + S;    // [S] MMA done with a stage
-  uint64_t* s_full = st_empty + S;     // S^T and dP^T in TMEM
-  uint64_t* ds_ready = s_full + 1;     // P^T and dS^T in TMEM (128 arrivals)
-  uint64_t* acc_done = ds_ready + 1;   // dK, dV final
+  uint8_t* sRing = smem + 2 * TB;  // stage s: Q_i at +0, dO_i at +TB
+  float* sLd = reinterpret_cast<float*>(smem + C::kSmemTiles);  // stage s: LSE2 [128], D [128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemTiles + C::kLdBytes);
+  uint64_t* kv_full = bars;           // K, V landed
+  uint64_t* st_full = bars + 1;       // [S] Q_i, dO_i, LSE2_i, D_i landed
+  uint64_t* st_empty = st_full + S;   // [S] MMA done with a stage
+  uint64_t* s_full = st_empty + S;    // S^T and dP^T in TMEM
+  uint64_t* ds_ready = s_full + 1;    // [4] quarter q of P^T and dS^T in TMEM (256 arrivals)
+  uint64_t* acc_done = ds_ready + 4;  // dK, dV final
   uint64_t* mma_done = acc_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -222,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&st_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(ds_ready, kElemThreads);
+    for (int q = 0; q < 4; ++q) mbar_init(&ds_ready[q], kElemThreads);
     mbar_init(acc_done, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -245,19 +323,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(sK + c * kChunkBytes, &tmK, kv_full, c * 64, j * kTile, bh);
         tma_load_3d(sV + c * kChunkBytes, &tmV, kv_full, c * 64, j * kTile, bh);
       }
+      const size_t ld_row = static_cast<size_t>(bh) * p.n_pad;
       int it = 0;
       for (; it < n_iter && ok; ++it) {
         const int s = it % S;
         const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
         ok = mbar_wait(&st_empty[s], ph ^ 1u, abort_flag, status, tmo, kSiteStage);
         if (!ok) break;
+        BWD_TRACE(0, 3, it, 0);
         const int i = i_first + it;
         uint8_t* st = sRing + s * C::kStageBytes;
-        mbar_arrive_expect_tx(&st_full[s], 2 * TB);
+        float* ld = sLd + s * 2 * kTile;
+        mbar_arrive_expect_tx(&st_full[s], 2 * TB + 2 * kTile * 4);
         for (int c = 0; c < C::kChunks; ++c) {
           tma_load_3d(st + c * kChunkBytes, &tmQ, &st_full[s], c * 64, i * kTile, bh);
           tma_load_3d(st + TB + c * kChunkBytes, &tmdO, &st_full[s], c * 64, i * kTile, bh);
         }
+        bulk_load(ld, p.lse2 + ld_row + i * kTile, kTile * 4, &st_full[s]);
+        bulk_load(ld + kTile, p.dd + ld_row + i * kTile, kTile * 4, &st_full[s]);
       }
       if (!ok) {
         for (int s = 0; s < S && s < it; ++s) {
@@ -281,10 +364,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                  kk > 0 ? 1u : 0u);
         }
       };
-      // acc (+)= A[tmem, 128 x 128 queries] * B[queries x d] (B MN-major)
-      auto issue_acc = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b, bool accumulate) {
+      // acc (+)= A[tmem, 128 x 32 queries of quarter q] * B[those queries x d] (B MN-major)
+      auto issue_acc_q = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b, int q, bool accumulate) {
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
+        for (int h = 0; h < 2; ++h) {
+          const int kk = 2 * q + h;
           mma_ts(d_tmem, a_tmem + packed_col(kk), sw128_desc(b + kk * 2048, kChunkBytes, 1024), idAcc,
                  (accumulate || kk > 0) ? 1u : 0u);
         }
@@ -292,84 +376,81 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(kv_full, 0, abort_flag, status, tmo, kSiteLoad);
       for (int it = 0; it < n_iter && ok; ++it) {
         const int s = it % S;
-        if (!(ok = mbar_wait(&st_full[s], static_cast<uint32_t>(it / S) & 1u, abort_flag, status, tmo, kSiteLoad))) break;
+        if (!(ok = mbar_wait(&st_full[s], static_cast<uint32_t>(it / S) & 1u, abort_flag, status, tmo, kSiteLoad)))
+          break;
+        BWD_TRACE(0, 0, it, 0);
         tc_fence_after();
         const uint32_t q = sr + s * C::kStageBytes, dO = q + TB;
         issue_abt(tmem + kColS, sk, q);   // S^T = K Q^T
         issue_abt(tmem + kColDP, sv, dO); // dP^T = V dO^T
         mma_commit(s_full);
-        if (!(ok = mbar_wait(ds_ready, static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteDs))) break;
-        tc_fence_after();
-        issue_acc(tmem + kColAcc, tmem + kColS, dO, it > 0);      // dV += P^T dO
-        issue_acc(tmem + kColAcc + D, tmem + kColDP, q, it > 0);  // dK += dS^T Q
+        BWD_TRACE(0, 0, it, 1);
+        for (int qq = 0; qq < 4 && ok; ++qq) {
+          if (!(ok = mbar_wait(&ds_ready[qq], static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteDs)))
+            break;
+          if (qq == 0) BWD_TRACE(0, 0, it, 2);
+          tc_fence_after();
+          issue_acc_q(tmem + kColAcc, tmem + kColS, dO, qq, it > 0);      // dV += P^T dO
+          issue_acc_q(tmem + kColAcc + D, tmem + kColDP, q, qq, it > 0);  // dK += dS^T Q
+        }
+        if (!ok) break;
         mma_commit(&st_empty[s]);
+        BWD_TRACE(0, 0, it, 3);
       }
       if (ok) mma_commit(acc_done);
       mma_commit(mma_done);
       mbar_wait_drain(mma_done, 0, tmo);
     }
   } else if (warp >= kElemWarp0) {
-    const int half = (warp - kElemWarp0) >> 2;  // which 64 of the 128 query columns
+    const int h = (warp - kElemWarp0) >> 2;  // which 16 columns of every quarter
     const int wq = warp & 3;
     const int r = wq * 32 + lane;  // key row inside the tile
     const int key = j * kTile + r;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_base + kColS, tDP = tmem + lane_base + kColDP;
     const float sl2 = p.scale_log2;
-    const float* lse_g = p.lse + static_cast<size_t>(bh) * p.N;
-    const float* d_g = p.dd + static_cast<size_t>(bh) * p.N;
-    // LSE (log2 units; first half of the threads) and D (second half) of the
-    // 128 queries of a tile, staged in shared memory (two buffers); queries
-    // past N get LSE = +inf, so P = 0 there.
-    auto fetch = [&](int i) {
-      const int qi = i * kTile + r;
-      if (half == 0) return qi < p.N ? lse_g[qi] * 1.4426950408889634f : INFINITY;
-      return qi < p.N ? d_g[qi] : 0.f;
-    };
-    float* stage_buf = half == 0 ? sLse : sD;
-    float nxt = n_iter > 0 ? fetch(i_first) : 0.f;
-    stage_buf[r] = nxt;
-    named_bar_sync(1, kElemThreads);
+    const bool tr = lane == 0 && wq == 0;
     bool ok = true;
-    for (int it = 0; it < n_iter; ++it) {
+    for (int it = 0; it < n_iter && ok; ++it) {
+      const int s = it % S;
       const int i = i_first + it;
-      const int buf = it & 1;
-      if (it + 1 < n_iter) nxt = fetch(i + 1);  // next tile's, early
-      const bool good = __all_sync(
-          0xffffffffu, mbar_wait(s_full, static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteS));
-      if (good) {
-        tc_fence_after();
-        const float* lt = sLse + buf * kTile;
-        const float* dt = sD + buf * kTile;
-        const bool diag = CAUSAL && i == j;
-        p_ds_tile<true>(
-            tS, tDP, 2 * half, sl2, [&](int c) { return lt[c]; }, [&](int c) { return dt[c]; },
-            [&](int c) { return !diag || i * kTile + c >= key; });
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(ds_ready);
-      }
-      stage_buf[(buf ^ 1) * kTile + r] = nxt;
-      // one barrier per iteration for every thread: it publishes the next
-      // tile's LSE/D and makes a give-up decision uniform across the warps
-      if (named_bar_or(1, kElemThreads, !good)) {
-        ok = false;
-        break;
-      }
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(s_full, static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteS));
+      // the stage's LSE2 and D come from the bulk copy engine: observe its barrier too
+      if (ok)
+        ok = __all_sync(0xffffffffu, mbar_wait(&st_full[s], static_cast<uint32_t>(it / S) & 1u, abort_flag,
+                                               status, tmo, kSiteLoad));
+      if (!ok) break;
+      if (tr) BWD_TRACE(0, 1 + h, it, 0);
+      tc_fence_after();
+      const float4* l4p = reinterpret_cast<const float4*>(sLd + s * 2 * kTile);
+      const float4* d4p = l4p + kTile / 4;
+      auto col = [&](int c, float4& l4, float4& d4) {
+        l4 = l4p[c >> 2];
+        d4 = d4p[c >> 2];
+      };
+      const int q0 = i * kTile;
+      auto allowed = [&](int c) { return q0 + c >= key; };
+      const bool diag = CAUSAL && i == j;
+      if (diag)
+        p_ds_tile<true, true>(tS, tDP, h, sl2, col, allowed, ds_ready);
+      else
+        p_ds_tile<true, false>(tS, tDP, h, sl2, col, allowed, ds_ready);
+      if (tr) BWD_TRACE(0, 1 + h, it, 1);
     }
     if (ok) ok = mbar_wait(acc_done, 0, abort_flag, status, tmo, kSiteO);
     const bool failed = named_bar_or(2, kElemThreads, !ok);
     if (!failed && n_iter > 0) {
       tc_fence_after();
-      // K and V are no longer read by any MMA: they stage dK (first half of
-      // the threads) and dV (second half)
-      if (half == 0)
+      // K and V are no longer read by any MMA: they stage dK (warps 4-7)
+      // and dV (warps 8-11)
+      if (h == 0)
         store_tile<D>(tmem + lane_base + kColAcc + D, p.scale, sK, r, 0, D / 32);
       else
         store_tile<D>(tmem + lane_base + kColAcc, 1.f, sV, r, 0, D / 32);
       fence_proxy_async_smem();
       named_bar_sync(1, kElemThreads);
-      if (half == 0 && r == 0) {
+      if (h == 0 && r == 0) {
         for (int c = 0; c < C::kChunks; ++c) {
           tma_store_3d(&tmdK, sK + c * kChunkBytes, c * 64, j * kTile, bh);
           tma_store_3d(&tmdV, sV + c * kChunkBytes, c * 64, j * kTile, bh);
@@ -390,19 +471,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// dQ: one CTA per query tile
+// dQ: one CTA per 128-query tile
 // ---------------------------------------------------------------------------
 template <int D>
 struct DqCfg {
   static constexpr int kChunks = D / 64;
   static constexpr int kTileBytes = kTile * D * 2;
-  static constexpr int kStages = D == 128 ? 2 : 3;      // each stage: K_j and V_j
+  static constexpr int kStages = D == 128 ? 2 : 4;  // each stage: K_j and V_j
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kSmemTiles = 2 * kTileBytes + kStages * kStageBytes;  // Q, dO, ring
-  static constexpr int kNumBars = 1 + 2 * kStages + 1 + 1 + 1 + 1;
+  static constexpr int kNumBars = 1 + 2 * kStages + 1 + 4 + 1 + 1;
   static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 1024;
 };
 
+// Same quarter pipeline over the key tiles j: S = Q K_j^T, dP = dO V_j^T, dS
+// in place a quarter (32 keys) at a time, dQ += dS K_j per quarter.
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -422,8 +505,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* st_full = bars + 1;
   uint64_t* st_empty = st_full + S;
   uint64_t* s_full = st_empty + S;
-  uint64_t* ds_ready = s_full + 1;
-  uint64_t* acc_done = ds_ready + 1;
+  uint64_t* ds_ready = s_full + 1;    // [4]
+  uint64_t* acc_done = ds_ready + 4;
   uint64_t* mma_done = acc_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -442,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&st_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(ds_ready, kElemThreads);
+    for (int q = 0; q < 4; ++q) mbar_init(&ds_ready[q], kElemThreads);
     mbar_init(acc_done, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -471,12 +554,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
         ok = mbar_wait(&st_empty[s], ph ^ 1u, abort_flag, status, tmo, kSiteStage);
         if (!ok) break;
-        const int jt = it;  // key tile
         uint8_t* st = sRing + s * C::kStageBytes;
         mbar_arrive_expect_tx(&st_full[s], 2 * TB);
         for (int c = 0; c < C::kChunks; ++c) {
-          tma_load_3d(st + c * kChunkBytes, &tmK, &st_full[s], c * 64, jt * kTile, bh);
-          tma_load_3d(st + TB + c * kChunkBytes, &tmV, &st_full[s], c * 64, jt * kTile, bh);
+          tma_load_3d(st + c * kChunkBytes, &tmK, &st_full[s], c * 64, it * kTile, bh);
+          tma_load_3d(st + TB + c * kChunkBytes, &tmV, &st_full[s], c * 64, it * kTile, bh);
         }
       }
       if (!ok) {
@@ -503,52 +585,72 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(q_full, 0, abort_flag, status, tmo, kSiteLoad);
       for (int it = 0; it < n_iter && ok; ++it) {
         const int s = it % S;
-        if (!(ok = mbar_wait(&st_full[s], static_cast<uint32_t>(it / S) & 1u, abort_flag, status, tmo, kSiteLoad))) break;
+        if (!(ok = mbar_wait(&st_full[s], static_cast<uint32_t>(it / S) & 1u, abort_flag, status, tmo, kSiteLoad)))
+          break;
+        BWD_TRACE(1, 0, it, 0);
         tc_fence_after();
         const uint32_t k = sr + s * C::kStageBytes, v = k + TB;
         issue_abt(tmem + kColS, sq, k);    // S = Q K^T
         issue_abt(tmem + kColDP, sdo, v);  // dP = dO V^T
         mma_commit(s_full);
-        if (!(ok = mbar_wait(ds_ready, static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteDs))) break;
-        tc_fence_after();
-        // dQ += dS K: A = dS in TMEM (over dP), B = K tile as [keys][d] (MN-major)
+        BWD_TRACE(1, 0, it, 1);
+        for (int qq = 0; qq < 4 && ok; ++qq) {
+          if (!(ok = mbar_wait(&ds_ready[qq], static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteDs)))
+            break;
+          if (qq == 0) BWD_TRACE(1, 0, it, 2);
+          tc_fence_after();
+          // dQ += dS K: A = dS in TMEM (over dP), B = K tile as [keys][d] (MN-major)
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          mma_ts(tmem + kColAcc, tmem + kColDP + packed_col(kk), sw128_desc(k + kk * 2048, kChunkBytes, 1024),
-                 idAcc, (it > 0 || kk > 0) ? 1u : 0u);
+          for (int hh = 0; hh < 2; ++hh) {
+            const int kk = 2 * qq + hh;
+            mma_ts(tmem + kColAcc, tmem + kColDP + packed_col(kk), sw128_desc(k + kk * 2048, kChunkBytes, 1024),
+                   idAcc, (it > 0 || kk > 0) ? 1u : 0u);
+          }
         }
+        if (!ok) break;
         mma_commit(&st_empty[s]);
+        BWD_TRACE(1, 0, it, 3);
       }
       if (ok) mma_commit(acc_done);
       mma_commit(mma_done);
       mbar_wait_drain(mma_done, 0, tmo);
     }
   } else if (warp >= kElemWarp0) {
-    const int half = (warp - kElemWarp0) >> 2;  // which 64 of the 128 key columns
+    const int h = (warp - kElemWarp0) >> 2;  // which 16 columns of every quarter
     const int wq = warp & 3;
     const int r = wq * 32 + lane;  // query row inside the tile
     const int row = i * kTile + r;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_base + kColS, tDP = tmem + lane_base + kColDP;
     const float sl2 = p.scale_log2;
-    // this row's LSE (log2 units) and D; rows past N get P = 0
-    const float lse2 = row < p.N ? p.lse[static_cast<size_t>(bh) * p.N + row] * 1.4426950408889634f : INFINITY;
-    const float dsub = row < p.N ? p.dd[static_cast<size_t>(bh) * p.N + row] : 0.f;
-    const int key_limit = CAUSAL ? min(row, p.N - 1) : p.N - 1;
+    const bool tr = lane == 0 && wq == 0;
+    // this row's LSE2 and D (padding rows: +inf and 0, so P = 0)
+    const size_t prow = static_cast<size_t>(bh) * p.n_pad + row;
+    const float lse2 = p.lse2[prow];
+    const float dsub = p.dd[prow];
+    const float4 l4c = make_float4(lse2, lse2, lse2, lse2);
+    const float4 d4c = make_float4(dsub, dsub, dsub, dsub);
+    auto col = [&](int, float4& l4, float4& d4) {
+      l4 = l4c;
+      d4 = d4c;
+    };
     bool ok = true;
     for (int it = 0; it < n_iter && ok; ++it) {
       ok = __all_sync(0xffffffffu,
                       mbar_wait(s_full, static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteS));
       if (!ok) break;
+      if (tr) BWD_TRACE(1, 1 + h, it, 0);
       tc_fence_after();
-      const int kbase = it * kTile;
-      const bool masked = (kbase + kTile > p.N) || (CAUSAL && kbase + kTile - 1 > i * kTile);
-      p_ds_tile<false>(
-          tS, tDP, 2 * half, sl2, [&](int) { return lse2; }, [&](int) { return dsub; },
-          [&](int c) { return !masked || kbase + c <= key_limit; });
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(ds_ready);
+      // keys past N need no mask: their K and V rows are zero, so they add
+      // nothing to dQ; the causal diagonal tile does
+      const int k0 = it * kTile;
+      auto allowed = [&](int c) { return k0 + c <= row; };
+      const bool diag = CAUSAL && it == i;
+      if (diag)
+        p_ds_tile<false, true>(tS, tDP, h, sl2, col, allowed, ds_ready);
+      else
+        p_ds_tile<false, false>(tS, tDP, h, sl2, col, allowed, ds_ready);
+      if (tr) BWD_TRACE(1, 1 + h, it, 1);
     }
     if (ok) ok = mbar_wait(acc_done, 0, abort_flag, status, tmo, kSiteO);
     const bool failed = named_bar_or(2, kElemThreads, !ok);
@@ -556,10 +658,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       // Q is no longer read by any MMA: it stages dQ, each half of the
       // threads taking half of the columns
-      store_tile<D>(tmem + lane_base + kColAcc, p.scale, sQ, r, half * (D / 64), (half + 1) * (D / 64));
+      store_tile<D>(tmem + lane_base + kColAcc, p.scale, sQ, r, h * (D / 64), (h + 1) * (D / 64));
       fence_proxy_async_smem();
       named_bar_sync(1, kElemThreads);
-      if (half == 0 && r == 0) {
+      if (h == 0 && r == 0) {
         for (int c = 0; c < C::kChunks; ++c) tma_store_3d(&tmdQ, sQ + c * kChunkBytes, c * 64, i * kTile, bh);
         bulk_commit_group();
         bulk_wait_group_read0();
@@ -600,7 +702,8 @@ fa_status set_smem(Kern kern, int bytes, int slot) {
 
 template <int D, bool CAUSAL>
 fa_status launch_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
-                     void* dQ, void* dK, void* dV, float* dd, BwdParams prm, cudaStream_t st) {
+                     const float* LSE, void* dQ, void* dK, void* dV, float* lse2, float* dd, BwdParams prm,
+                     cudaStream_t st) {
   const int N = prm.N, BH = prm.BH;
   CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv;
   if (!host::make_map(&mq, Q, D, N, BH, kTile) || !host::make_map(&mk, K, D, N, BH, kTile) ||
@@ -610,9 +713,10 @@ fa_status launch_bwd(const void* Q, const void* K, const void* V, const void* O,
     snprintf(host::g_last_error, sizeof(host::g_last_error), "cuTensorMapEncodeTiled failed");
     return FA_ERR_CUDA;
   }
-  const long long rows = static_cast<long long>(BH) * N;
-  bwd_rowdot_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), dd, rows);
+  const long long rows_pad = static_cast<long long>(BH) * prm.n_pad;
+  bwd_rowdot_kernel<D><<<static_cast<unsigned>((rows_pad + 7) / 8), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), LSE, lse2, dd, N,
+      prm.n_pad, rows_pad);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return host::cuda_fail(e, "bwd rowdot launch");
   const unsigned grid = static_cast<unsigned>(static_cast<long long>(BH) * prm.n_tiles);
@@ -647,9 +751,18 @@ cudaError_t read_and_clear_status(uint32_t* v) {
 
 extern "C" {
 
+#ifdef FA_TRACE
+// Trace builds only: device buffer of 2*16*4*64*8 uint64 (or NULL).
+int fa_bwd_trace_set(void* device_buffer) {
+  return cudaMemcpyToSymbol(fa::bwd::g_bwd_trace, &device_buffer, sizeof(device_buffer)) == cudaSuccess ? 0 : 1;
+}
+#endif
+
 size_t fa_bwd_workspace_bytes(int B, int H, int N) {
   if (B < 1 || H < 1 || N < 1) return 0;
-  return static_cast<size_t>(B) * H * N * 4;
+  // LSE * log2(e) and D = rowsum(dO * O), fp32, each [B][H][N rounded up to 128]
+  const size_t n_pad = (static_cast<size_t>(N) + fa::bwd::kTile - 1) / fa::bwd::kTile * fa::bwd::kTile;
+  return 2 * static_cast<size_t>(B) * H * n_pad * 4;
 }
 
 fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
@@ -685,11 +798,14 @@ fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, con
   fa_status st0 = host::require_sm100();
   if (st0 != FA_OK) return st0;
   bwd::BwdParams prm{};
-  prm.lse = LSE;
-  prm.dd = static_cast<const float*>(workspace);
   prm.N = N;
-  prm.BH = static_cast<int>(BH);
   prm.n_tiles = static_cast<int>(n_tiles);
+  prm.n_pad = prm.n_tiles * bwd::kTile;
+  prm.BH = static_cast<int>(BH);
+  float* lse2 = static_cast<float*>(workspace);
+  float* dd = lse2 + static_cast<size_t>(BH) * prm.n_pad;
+  prm.lse2 = lse2;
+  prm.dd = dd;
   {
     // keep the Q, dO, K, V of one group of heads (8*N*d bytes per head) within ~48 MB of L2
     const long long per_head = 8ll * N * d;
@@ -700,12 +816,11 @@ fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, con
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
   prm.timeout_ns = host::wait_timeout_ns();
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float* dd = static_cast<float*>(workspace);
   if (d == 128)
-    return causal ? bwd::launch_bwd<128, true>(Q, K, V, O, dO, dQ, dK, dV, dd, prm, st)
-                  : bwd::launch_bwd<128, false>(Q, K, V, O, dO, dQ, dK, dV, dd, prm, st);
-  return causal ? bwd::launch_bwd<64, true>(Q, K, V, O, dO, dQ, dK, dV, dd, prm, st)
-                : bwd::launch_bwd<64, false>(Q, K, V, O, dO, dQ, dK, dV, dd, prm, st);
+    return causal ? bwd::launch_bwd<128, true>(Q, K, V, O, dO, LSE, dQ, dK, dV, lse2, dd, prm, st)
+                  : bwd::launch_bwd<128, false>(Q, K, V, O, dO, LSE, dQ, dK, dV, lse2, dd, prm, st);
+  return causal ? bwd::launch_bwd<64, true>(Q, K, V, O, dO, LSE, dQ, dK, dV, lse2, dd, prm, st)
+                : bwd::launch_bwd<64, false>(Q, K, V, O, dO, LSE, dQ, dK, dV, lse2, dd, prm, st);
 }
 
 }  // extern "C"

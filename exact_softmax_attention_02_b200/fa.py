@@ -260,6 +260,11 @@ def fa_fwd_block_sparse(q, k, v, o, row_ptr, col_idx, lse=None, scale: float | N
                                    _stream_handle(stream)))
 
 
+def bwd_workspace_bytes(B: int, H: int, N: int) -> int:
+    """Workspace bytes fa_bwd needs."""
+    return int(_load().fa_bwd_workspace_bytes(B, H, N))
+
+
 def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace=None, scale: float | None = None,
            causal: bool = False, stream=None) -> None:
     """Backward pass: dq, dk, dv of L = sum(o * do) for o = fa_fwd(q, k, v).

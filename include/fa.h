@@ -125,7 +125,8 @@ int fa_fwd_splitkv_default_splits(int B, int H, int N, int d, int causal);
  *   LSE             device, fp32 [B][H][N], read (as written by fa_fwd).
  *   dQ, dK, dV      device, bf16 [B][H][N][d], written.
  *   workspace       device, 16-byte aligned, >= fa_bwd_workspace_bytes(B, H,
- *                   N) bytes, overwritten (D, fp32 [B][H][N]).
+ *                   N) bytes, overwritten: LSE * log2(e) and D, each fp32
+ *                   [B][H][N rounded up to 128].
  *   B, H, N, d, scale, causal, stream: as for fa_fwd.
  * The outputs and the workspace must not overlap the inputs or each other.
  * Three kernels are enqueued on `stream`.  Errors as fa_fwd, plus
@@ -137,7 +138,8 @@ fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, con
                  size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
                  void* stream);
 
-/* Bytes of workspace fa_bwd needs (0 for invalid arguments). */
+/* Bytes of workspace fa_bwd needs: 8 * B * H * (N rounded up to 128); 0 for
+ * invalid arguments. */
 size_t fa_bwd_workspace_bytes(int B, int H, int N);
 
 /* Size of the workspace built into the library for fa_fwd_splitkv_noalloc. */

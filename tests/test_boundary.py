@@ -160,7 +160,8 @@ def test_bwd_argument_checks(lib):
     lib.fa_bwd.restype = ci
     lib.fa_bwd_workspace_bytes.argtypes = [ci, ci, ci]
     lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
-    assert lib.fa_bwd_workspace_bytes(2, 3, 100) == 2 * 3 * 100 * 4
+    assert lib.fa_bwd_workspace_bytes(2, 3, 100) == 2 * 2 * 3 * 128 * 4
+    assert lib.fa_bwd_workspace_bytes(1, 1, 129) == 2 * 256 * 4
     base = [A + k * 64 * MB for k in range(10)]  # Q K V O dO LSE dQ dK dV ws
 
     def bwd(args=None, ws_bytes=1 << 20, N=128, d=64):
@@ -173,7 +174,7 @@ def test_bwd_argument_checks(lib):
         assert bwd(a) == FA_ERR_NULL
     assert bwd(d=96) == FA_ERR_UNSUPPORTED
     assert bwd(N=0) == FA_ERR_SHAPE
-    assert bwd(ws_bytes=128 * 4 - 4) == FA_ERR_WORKSPACE
+    assert bwd(ws_bytes=2 * 128 * 4 - 4) == FA_ERR_WORKSPACE
     a = list(base)
     a[6] = base[0] + 32  # dQ overlapping Q
     assert bwd(a) == FA_ERR_ALIAS
