@@ -207,7 +207,8 @@ def committed_traffic(workload: str):
             line = line.strip().lstrip("-* ")
             for key in ("dram_bytes_per_launch", "kernel_source_sha256"):
                 if line.startswith(key + ":"):
-                    vals[key] = line.split(":", 1)[1].strip().strip("`")
+                    rest = line.split(":", 1)[1].split()
+                    vals[key] = rest[0].strip("`") if rest else ""
     if vals.get("kernel_source_sha256") != kernel_source_hash():
         return None
     try:

@@ -2,9 +2,10 @@
 
     python -m exact_softmax_attention_02_b200.build [--force] [--verbose]
 
-The library is built from csrc/fa_fwd.cu (the fused forward, split-KV and
-merge), csrc/fa_bwd.cu (the backward pass) and csrc/standard_softmax.cu (the
-comparator's softmax), linked
+The library is built from csrc/fa_fwd.cu (the fused forward, split-KV,
+merge, block-sparse and key-tile variants), csrc/fa_bwd.cu (the backward
+pass), csrc/fa_host.cu (the host-buffer forward with pipelined copies) and
+csrc/standard_softmax.cu (the comparator's softmax), linked
 against the static CUDA runtime; the driver entry point for tensor-map encoding is looked
 up at run time, so no libcuda link is needed.
 """
@@ -19,7 +20,8 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = [os.path.join(HERE, "csrc", n) for n in ("fa_fwd.cu", "fa_bwd.cu", "standard_softmax.cu")]
+SOURCES = [os.path.join(HERE, "csrc", n)
+           for n in ("fa_fwd.cu", "fa_bwd.cu", "fa_host.cu", "standard_softmax.cu")]
 DEPENDS = SOURCES + [os.path.join(HERE, "csrc", "sm100.cuh"), os.path.join(HERE, "csrc", "host_util.h"),
                      os.path.join(ROOT, "include", "fa.h")]
 OUTPUT = os.path.join(HERE, "libfa.so")

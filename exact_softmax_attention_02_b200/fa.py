@@ -81,6 +81,11 @@ def _load():
     lib.fa_fwd_key_tile.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_float, c_int, c_int,
                                     vp]
     lib.fa_fwd_key_tile.restype = c_int
+    lib.fa_fwd_host.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_size_t, c_int, c_int, c_int, c_int, c_float,
+                                c_int, c_int, vp]
+    lib.fa_fwd_host.restype = c_int
+    lib.fa_fwd_host_workspace_bytes.argtypes = [c_int, c_int, c_int, c_int]
+    lib.fa_fwd_host_workspace_bytes.restype = ctypes.c_size_t
     lib.fa_version.argtypes = []
     lib.fa_version.restype = ctypes.c_char_p
     _lib = lib
@@ -292,20 +297,89 @@ def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace=None, scale: float | None 
                       B, H, N, d, float(scale), int(bool(causal)), _stream_handle(stream)))
 
 
+def host_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    """Device workspace bytes fa_fwd_host needs."""
+    return int(_load().fa_fwd_host_workspace_bytes(B, H, N, d))
+
+
+def fa_fwd_host(q, k, v, o, lse=None, workspace=None, chunks: int = 0, scale: float | None = None,
+                causal: bool = False, stream=None) -> None:
+    """The forward on HOST tensors, copies pipelined with the kernels (fa_fwd_host).
+
+    q, k, v, o: CPU bf16 [B, H, N, d] contiguous (pinned for overlapping
+    copies); lse: CPU float32 [B, H, N] or None.  ``workspace``: a CUDA
+    tensor of at least host_workspace_bytes(...) bytes on the device to run
+    on.  Asynchronous on ``stream``: synchronise it before reading o and lse.
+    """
+    lib = _load()
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        if t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous CPU bfloat16 [B, H, N, d] tensor")
+    if not (q.shape == k.shape == v.shape == o.shape):
+        raise ValueError("q, k, v, o must have the same shape")
+    B, H, N, d = q.shape
+    lse_ptr = None
+    if lse is not None:
+        if lse.dtype != torch.float32 or lse.is_cuda or not lse.is_contiguous() or tuple(lse.shape) != (B, H, N):
+            raise ValueError(f"lse must be a contiguous CPU float32 [B, H, N] = {(B, H, N)} tensor")
+        lse_ptr = lse.data_ptr()
+    if workspace is None or not workspace.is_cuda:
+        raise ValueError("workspace must be a CUDA tensor")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    _check(lib.fa_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_ptr,
+                           workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                           B, H, N, d, float(scale), int(bool(causal)), int(chunks),
+                           _stream_handle(stream)))
+
+
+_host_workspaces = {}
+
+
+def _host_workspace(device: torch.device, nbytes: int) -> torch.Tensor:
+    """A device workspace of at least ``nbytes``, kept per device for reuse."""
+    ws = _host_workspaces.get(device)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+        _host_workspaces[device] = ws
+    return ws
+
+
 def attention_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                       scale: float | None = None, causal: bool = False,
                       return_lse: bool = True, device=None, out=None, num_splits=None):
     """Allocate the outputs and run the forward.
 
     CUDA inputs: outputs stay on their device.  CPU inputs (ideally pinned):
-    they are copied to ``device`` (default: the current CUDA device), the
-    kernel runs there, and O (and LSE) are copied back to host memory -- into
-    ``out = (o_host, lse_host)`` when given (pinned buffers of the right shape
-    and dtype, reused across calls), else into new pinned tensors.  The call
-    returns after the copies have completed.  ``num_splits`` (not None) runs
-    the split-KV forward with that many key ranges (0: its default).
+    fa_fwd_host copies them to ``device`` (default: the current CUDA device)
+    and O (and LSE) back to host memory, pipelined with the kernels over
+    groups of heads -- into ``out = (o_host, lse_host)`` when given (pinned
+    buffers of the right shape and dtype, reused across calls), else into new
+    pinned tensors.  The call returns after the copies have completed.
+    ``num_splits`` (not None) runs the split-KV forward with that many key
+    ranges (0: its default), with whole-tensor copies.
     """
     on_host = not q.is_cuda
+    if on_host and num_splits is None:
+        dev = torch.device(device) if device is not None else torch.device(
+            "cuda", torch.cuda.current_device())
+        if out is not None:
+            o_h, lse_h = out
+            if tuple(o_h.shape) != tuple(q.shape) or o_h.dtype != q.dtype:
+                raise ValueError("out[0] must match q in shape and dtype")
+            if return_lse and (lse_h is None or tuple(lse_h.shape) != tuple(q.shape[:3])):
+                raise ValueError("out[1] must be a float32 [B, H, N] tensor")
+        else:
+            o_h = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+            lse_h = torch.empty(q.shape[:3], dtype=torch.float32, pin_memory=True) if return_lse else None
+        B, H, N, d = q.shape
+        with torch.cuda.device(dev):
+            ws = _host_workspace(dev, host_workspace_bytes(B, H, N, d))
+            stream = torch.cuda.current_stream(dev)
+            fa_fwd_host(q.contiguous(), k.contiguous(), v.contiguous(), o_h, lse_h if return_lse else None,
+                        workspace=ws, scale=scale, causal=causal, stream=stream)
+            stream.synchronize()
+        return (o_h, lse_h) if return_lse else o_h
     if on_host:
         dev = torch.device(device) if device is not None else torch.device(
             "cuda", torch.cuda.current_device())

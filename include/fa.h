@@ -190,6 +190,40 @@ fa_status fa_fwd_splitkv_noalloc(const void* Q, const void* K, const void* V, vo
 fa_status fa_fwd_key_tile(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
                           int H, int N, int d, float scale, int causal, int key_tile, void* stream);
 
+/*
+ * fa_fwd_host -- fa_fwd on inputs and outputs in HOST memory: the end-to-end
+ * call.  Q, K, V are copied to the device, the forward runs there, and O and
+ * LSE are copied back, all pipelined over `chunks` groups of heads on three
+ * streams of the library's own.  While one group is copied in, the previous
+ * one is computed and the one before is copied out.  Each (b, h) pair needs
+ * only its own Q, K, V (lihaoran.work, the opening formula), so the split
+ * does not change any output bit.
+ *
+ *   Qh, Kh, Vh   host, bf16 [B][H][N][d], read.  Pinned memory
+ *                (cudaHostAlloc / cudaHostRegister) lets the copies overlap;
+ *                pageable memory works but serialises them.
+ *   Oh           host, bf16 [B][H][N][d], written.
+ *   LSEh         host, fp32 [B][H][N], written; may be NULL.
+ *   workspace    device, 16-byte aligned, >= fa_fwd_host_workspace_bytes(B,
+ *                H, N, d) bytes: the device copies of Q, K, V, O, LSE.
+ *   chunks       groups of heads (<= 0: 8; capped at B*H and 64).
+ *   B, H, N, d, scale, causal: as fa_fwd.
+ *   stream       the caller's stream: the work starts after what is already
+ *                queued on it, and work queued on it afterwards waits until
+ *                O and LSE have reached host memory.  Synchronise it before
+ *                reading them.
+ * The first call on a device creates the library's three streams and its
+ * events (no device memory).  Errors: as fa_fwd, plus FA_ERR_WORKSPACE for a
+ * short workspace and FA_ERR_UNSUPPORTED when a host argument is device or
+ * managed memory or the workspace is not device memory.
+ */
+fa_status fa_fwd_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, float* LSEh,
+                      void* workspace, size_t workspace_bytes, int B, int H, int N, int d, float scale,
+                      int causal, int chunks, void* stream);
+
+/* Device workspace bytes fa_fwd_host needs: 8*B*H*N*d + 4*B*H*N (0 if invalid). */
+size_t fa_fwd_host_workspace_bytes(int B, int H, int N, int d);
+
 /* Block of the block-sparse layout: query rows x keys. */
 #define FA_BLOCK_Q 256
 #define FA_BLOCK_K 128

@@ -222,3 +222,27 @@ def test_key_tile_argument_checks(lib):
     assert kt(64, q=None) == FA_ERR_NULL
     assert kt(64, d=32) == FA_ERR_UNSUPPORTED
     assert kt(128, q=A + 8) == FA_ERR_ALIGN
+
+
+def test_host_forward_argument_checks(lib):
+    vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.fa_fwd_host.argtypes = [vp] * 6 + [ctypes.c_size_t] + [ci] * 4 + [cf, ci, ci, vp]
+    lib.fa_fwd_host.restype = ci
+    lib.fa_fwd_host_workspace_bytes.argtypes = [ci] * 4
+    lib.fa_fwd_host_workspace_bytes.restype = ctypes.c_size_t
+    need = lib.fa_fwd_host_workspace_bytes(2, 3, 100, 64)
+    assert need == 4 * 2 * 3 * 100 * 64 * 2 + 2 * 3 * 100 * 4
+    assert lib.fa_fwd_host_workspace_bytes(1, 1, 100, 96) == 0
+    ws = A + 512 * MB
+
+    def fh(q=A, ws=ws, ws_bytes=1 << 30, N=1024, d=64, scale=0.125):
+        return lib.fa_fwd_host(q, A + 64 * MB, A + 128 * MB, A + 192 * MB, A + 256 * MB, ws, ws_bytes,
+                               1, 1, N, d, scale, 0, 0, None)
+
+    assert fh(q=None) == FA_ERR_NULL
+    assert fh(ws=None) == FA_ERR_NULL
+    assert fh(N=0) == FA_ERR_SHAPE
+    assert fh(d=96) == FA_ERR_UNSUPPORTED
+    assert fh(scale=-1.0) == FA_ERR_UNSUPPORTED
+    assert fh(ws=ws + 8) == FA_ERR_ALIGN
+    assert fh(ws_bytes=lib.fa_fwd_host_workspace_bytes(1, 1, 1024, 64) - 4) == FA_ERR_WORKSPACE

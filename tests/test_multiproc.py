@@ -79,3 +79,22 @@ def test_reference_arm_under_torchrun_prints_once():
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["value"] > 0 and line["unit"] == "TFLOP/s"
+
+
+def test_committed_traffic_reads_the_profile_summary(tmp_path, monkeypatch):
+    """The bench reports DRAM traffic from the committed ncu summary only while its
+    kernel source hash matches the current sources."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "KERNEL_SOURCES", [])  # the hash of no sources
+    (prof / "fa_fwd_wl_ncu.md").write_text(
+        "- kernel_source_sha256: `%s` (note)\n- dram_bytes_per_launch: 1234\n" % bench.kernel_source_hash())
+    (prof / "fa_fwd_old_ncu.md").write_text(
+        "- kernel_source_sha256: `0000000000000000` (note)\n- dram_bytes_per_launch: 99\n")
+    assert bench.committed_traffic("wl") == 1234.0
+    assert bench.committed_traffic("old") is None
+    assert bench.committed_traffic("missing") is None
