@@ -379,7 +379,7 @@ def run_ours(args, w):
     if fa.device_status(stream) != 0:
         raise RuntimeError("kernel reported a device timeout during warm-up")
 
-    sampler = ClockSampler(local_rank, period_s=float(os.environ.get("FA_BENCH_CLOCK_PERIOD", "0.05")))
+    sampler = ClockSampler(local_rank, period_s=float(os.environ.get("FA_BENCH_CLOCK_PERIOD", "0.01")))
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -483,6 +483,9 @@ def run_ours(args, w):
                     "kernel": "fa_std::softmax_rows_kernel", "algorithmic_bytes": nbytes,
                     "step_tflops": achieved}
     launches = int(sum_over_ranks(args.steps * launches_per_step, dist, dev))
+    srt = sorted(launch_ms)
+    step_ms = {"min": srt[0], "median": srt[len(srt) // 2], "max": srt[-1],
+               "first5_mean": sum(launch_ms[:5]) / min(5, len(launch_ms))}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and bwd is None:
@@ -508,6 +511,7 @@ def run_ours(args, w):
             "e2e": {"value": weak_scaling_value(flops, world, e2e_steps, e2e_s), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
+            "step_ms": step_ms,
             "clocks": clocks,
             "cpu_baseline": cpu,
         }
