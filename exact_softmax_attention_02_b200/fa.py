@@ -106,63 +106,6 @@ def _stream_handle(stream) -> int:
     return int(stream.cuda_stream)
 
 
-def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
-           lse: torch.Tensor | None = None, scale: float | None = None,
-           causal: bool = False, stream=None) -> None:
-    """Launch the fused forward: o = softmax(scale q k^T [causal]) v, lse.
-
-    q, k, v, o: CUDA bfloat16 [B, H, N, d], contiguous (d = 64 or 128).
-    lse: CUDA float32 [B, H, N] contiguous, or None.
-    scale: defaults to 1/sqrt(d).  Asynchronous on ``stream`` (default: the
-    current stream).
-    """
-    lib = _load()
-    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
-        if t.dtype != torch.bfloat16:
-            raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
-        if not t.is_cuda:
-            raise ValueError(f"{name} must be a CUDA tensor")
-        if not t.is_contiguous():
-            raise ValueError(f"{name} must be contiguous")
-        if t.dim() != 4:
-            raise ValueError(f"{name} must be [B, H, N, d]")
-    if not (q.shape == k.shape == v.shape == o.shape):
-        raise ValueError(f"shape mismatch: q{tuple(q.shape)} k{tuple(k.shape)} "
-                         f"v{tuple(v.shape)} o{tuple(o.shape)}")
-    B, H, N, d = q.shape
-    lse_ptr = None
-    if lse is not None:
-        if lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous():
-            raise ValueError("lse must be a contiguous CUDA float32 tensor")
-        if tuple(lse.shape) != (B, H, N):
-            raise ValueError(f"lse must be [B, H, N] = {(B, H, N)}")
-        lse_ptr = lse.data_ptr()
-    if scale is None:
-        scale = 1.0 / math.sqrt(d)
-    _check(lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_ptr,
-                      B, H, N, d, float(scale), int(bool(causal)), _stream_handle(stream)))
-
-
-def fa_fwd_key_tile(q, k, v, o, lse=None, key_tile: int = 128, scale: float | None = None,
-                    causal: bool = False, stream=None) -> None:
-    """fa_fwd on 128 x ``key_tile`` score tiles (64 or 128), for the tile-size sweep."""
-    lib = _load()
-    _check_qkvo(q, k, v, o)
-    B, H, N, d = q.shape
-    lse_ptr = None
-    if lse is not None:
-        if lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous():
-            raise ValueError("lse must be a contiguous CUDA float32 tensor")
-        if tuple(lse.shape) != (B, H, N):
-            raise ValueError(f"lse must be [B, H, N] = {(B, H, N)}")
-        lse_ptr = lse.data_ptr()
-    if scale is None:
-        scale = 1.0 / math.sqrt(d)
-    _check(lib.fa_fwd_key_tile(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_ptr,
-                               B, H, N, d, float(scale), int(bool(causal)), int(key_tile),
-                               _stream_handle(stream)))
-
-
 def _check_qkvo(q, k, v, o):
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
         if t.dtype != torch.bfloat16:
@@ -176,6 +119,69 @@ def _check_qkvo(q, k, v, o):
     if not (q.shape == k.shape == v.shape == o.shape):
         raise ValueError(f"shape mismatch: q{tuple(q.shape)} k{tuple(k.shape)} "
                          f"v{tuple(v.shape)} o{tuple(o.shape)}")
+
+
+def _lse_ptr(lse, B: int, H: int, N: int):
+    """Pointer of an optional fp32 [B, H, N] CUDA tensor (None -> NULL)."""
+    if lse is None:
+        return None
+    if lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous CUDA float32 tensor")
+    if tuple(lse.shape) != (B, H, N):
+        raise ValueError(f"lse must be [B, H, N] = {(B, H, N)}")
+    return lse.data_ptr()
+
+
+def _launch_device(stream, *tensors) -> torch.device:
+    """The one CUDA device every tensor (and the stream, if given) lives on.
+
+    The kernels run on the current device and dereference every pointer there,
+    so tensors spread over several devices are refused here."""
+    devs = {t.device for t in tensors if t is not None}
+    if len(devs) != 1:
+        raise ValueError(f"all tensors must be on one CUDA device, got {sorted(str(d) for d in devs)}")
+    dev = devs.pop()
+    if stream is not None and stream.device != dev:
+        raise ValueError(f"stream is on {stream.device}, tensors on {dev}")
+    return dev
+
+
+def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+           lse: torch.Tensor | None = None, scale: float | None = None,
+           causal: bool = False, stream=None) -> None:
+    """Launch the fused forward: o = softmax(scale q k^T [causal]) v, lse.
+
+    q, k, v, o: CUDA bfloat16 [B, H, N, d], contiguous (d = 64 or 128), on one
+    device.  lse: CUDA float32 [B, H, N] contiguous, or None.
+    scale: defaults to 1/sqrt(d).  Asynchronous on ``stream`` (default: the
+    current stream of the tensors' device).
+    """
+    lib = _load()
+    _check_qkvo(q, k, v, o)
+    B, H, N, d = q.shape
+    lse_ptr = _lse_ptr(lse, B, H, N)
+    dev = _launch_device(stream, q, k, v, o, lse)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    with torch.cuda.device(dev):
+        _check(lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_ptr,
+                          B, H, N, d, float(scale), int(bool(causal)), _stream_handle(stream)))
+
+
+def fa_fwd_key_tile(q, k, v, o, lse=None, key_tile: int = 128, scale: float | None = None,
+                    causal: bool = False, stream=None) -> None:
+    """fa_fwd on 128 x ``key_tile`` score tiles (64 or 128), for the tile-size sweep."""
+    lib = _load()
+    _check_qkvo(q, k, v, o)
+    B, H, N, d = q.shape
+    lse_ptr = _lse_ptr(lse, B, H, N)
+    dev = _launch_device(stream, q, k, v, o, lse)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    with torch.cuda.device(dev):
+        _check(lib.fa_fwd_key_tile(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_ptr,
+                                   B, H, N, d, float(scale), int(bool(causal)), int(key_tile),
+                                   _stream_handle(stream)))
 
 
 def splitkv_workspace_bytes(B: int, H: int, N: int, d: int, num_splits: int = 0,
@@ -195,24 +201,20 @@ def fa_fwd_splitkv(q, k, v, o, lse=None, workspace=None, num_splits: int = 0,
     lib = _load()
     _check_qkvo(q, k, v, o)
     B, H, N, d = q.shape
-    lse_ptr = None
-    if lse is not None:
-        if lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous():
-            raise ValueError("lse must be a contiguous CUDA float32 tensor")
-        if tuple(lse.shape) != (B, H, N):
-            raise ValueError(f"lse must be [B, H, N] = {(B, H, N)}")
-        lse_ptr = lse.data_ptr()
+    lse_ptr = _lse_ptr(lse, B, H, N)
     if workspace is None:
         nbytes = splitkv_workspace_bytes(B, H, N, d, num_splits, causal)
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
     if not workspace.is_cuda or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
+    dev = _launch_device(stream, q, k, v, o, lse, workspace)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    _check(lib.fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_ptr,
-                              workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                              B, H, N, d, float(scale), int(bool(causal)), int(num_splits),
-                              _stream_handle(stream)))
+    with torch.cuda.device(dev):
+        _check(lib.fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_ptr,
+                                  workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                  B, H, N, d, float(scale), int(bool(causal)), int(num_splits),
+                                  _stream_handle(stream)))
 
 
 def block_layout_to_csr(layout, device=None):
@@ -249,20 +251,16 @@ def fa_fwd_block_sparse(q, k, v, o, row_ptr, col_idx, lse=None, scale: float | N
             raise ValueError(f"{name} must be a contiguous 1-D CUDA int32 tensor")
     if row_ptr.numel() != n_qb + 1:
         raise ValueError(f"row_ptr must have ceil(N / {BLOCK_Q}) + 1 = {n_qb + 1} entries")
-    lse_ptr = None
-    if lse is not None:
-        if lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous():
-            raise ValueError("lse must be a contiguous CUDA float32 tensor")
-        if tuple(lse.shape) != (B, H, N):
-            raise ValueError(f"lse must be [B, H, N] = {(B, H, N)}")
-        lse_ptr = lse.data_ptr()
+    lse_ptr = _lse_ptr(lse, B, H, N)
+    dev = _launch_device(stream, q, k, v, o, lse, row_ptr, col_idx)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     nnz = col_idx.numel()
-    _check(lib.fa_fwd_block_sparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_ptr,
-                                   row_ptr.data_ptr(), col_idx.data_ptr() if nnz else None, nnz,
-                                   B, H, N, d, float(scale), int(bool(causal)),
-                                   _stream_handle(stream)))
+    with torch.cuda.device(dev):
+        _check(lib.fa_fwd_block_sparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_ptr,
+                                       row_ptr.data_ptr(), col_idx.data_ptr() if nnz else None, nnz,
+                                       B, H, N, d, float(scale), int(bool(causal)),
+                                       _stream_handle(stream)))
 
 
 def bwd_workspace_bytes(B: int, H: int, N: int) -> int:
@@ -284,17 +282,22 @@ def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace=None, scale: float | None 
     if do.shape != q.shape:
         raise ValueError("do, dq, dk, dv must have the shape of q")
     B, H, N, d = q.shape
-    if lse.dtype != torch.float32 or not lse.is_cuda or tuple(lse.shape) != (B, H, N):
-        raise ValueError(f"lse must be a CUDA float32 [B, H, N] = {(B, H, N)} tensor")
+    if lse is None:
+        raise ValueError("lse (the forward's) is required")
+    lse_ptr = _lse_ptr(lse, B, H, N)
     need = int(lib.fa_bwd_workspace_bytes(B, H, N))
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    dev = _launch_device(stream, q, k, v, o, do, lse, dq, dk, dv, workspace)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    _check(lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
-                      lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                      workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                      B, H, N, d, float(scale), int(bool(causal)), _stream_handle(stream)))
+    with torch.cuda.device(dev):
+        _check(lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                          lse_ptr, dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                          workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                          B, H, N, d, float(scale), int(bool(causal)), _stream_handle(stream)))
 
 
 def host_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
@@ -325,12 +328,14 @@ def fa_fwd_host(q, k, v, o, lse=None, workspace=None, chunks: int = 0, scale: fl
         lse_ptr = lse.data_ptr()
     if workspace is None or not workspace.is_cuda:
         raise ValueError("workspace must be a CUDA tensor")
+    dev = _launch_device(stream, workspace)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    _check(lib.fa_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_ptr,
-                           workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                           B, H, N, d, float(scale), int(bool(causal)), int(chunks),
-                           _stream_handle(stream)))
+    with torch.cuda.device(dev):
+        _check(lib.fa_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_ptr,
+                               workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                               B, H, N, d, float(scale), int(bool(causal)), int(chunks),
+                               _stream_handle(stream)))
 
 
 _host_workspaces = {}
