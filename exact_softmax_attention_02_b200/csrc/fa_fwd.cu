@@ -78,7 +78,8 @@ static_assert(kEmuPer32 >= 0 && kEmuPer32 <= 32 && kEmuPer32 % 2 == 0, "even cou
 #define FA_P_HALVES 1
 #endif
 // 1: P_t is published once per tile; 2: in two halves of 64 keys, each on its
-// own barrier, so that the PV product can start on the first half
+// own barrier, so that the PV product can start on the first half (128-key
+// tiles only; 64-key tiles always publish P whole)
 constexpr int kPHalves = FA_P_HALVES;
 static_assert(kPHalves == 1 || kPHalves == 2, "P is published whole or in two halves");
 constexpr uint32_t kTmemCols = 512;
@@ -95,7 +96,7 @@ struct FwdParams {
   int BH;               // batch * heads
   int group_heads;      // heads whose CTAs are scheduled together
   int n_qblk;           // ceil(N / 256)
-  int n_kv;             // ceil(N / 128)
+  int n_kv;             // ceil(N / key tile)
   float scale_log2;     // scale * log2(e)
   uint64_t timeout_ns;  // bound on every wait
   uint32_t debug;       // bit 0: stall the softmax warps on a barrier nobody signals
@@ -170,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int S = C::kStages;
   constexpr int QB = C::kQBytes;
   static_assert(BN == BN || !(SPLIT || SPARSE), "split-KV and block-sparse use 128-key tiles");
-  static_assert(BN == 128 || kPHalves == 1, "P is published in halves only with 128-key tiles");
+  constexpr int kPH = BN == 128 ? kPHalves : 1;  // P publications per tile
   constexpr int SB = C::kStageBytes;
   static_assert(!PAIR || D == 128, "the pair kernel splits d = 128 into two 64-wide halves");
   static_assert(!(PAIR && SPLIT), "split-KV uses the single-CTA shape");
@@ -429,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool k_ready = false;
         for (int t = 0; t < 2; ++t) {
           if (it >= first_it[t]) {
-            // P_t arrives whole on p_half[2t], or (kPHalves == 2) in two
+            // P_t arrives whole on p_half[2t], or (kPH == 2) in two
             // halves of 64 keys on p_half[2t] and p_half[2t+1], so that the
             // first four K-steps of the PV product start while the softmax
             // is still on the second half.
@@ -439,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             FA_TRACE_MARK(0, it, 3 * t);
             tc_fence_after();
             issue_pv(t, sv, acc, 0);
-            if (kPHalves == 2 &&
+            if (kPH == 2 &&
                 !(ok = mbar_wait<PAIR>(&p_half[2 * t + 1], ph, abort_flag, status, tmo, kSiteP + 2 * t + 1))) break;
             tc_fence_after();
             issue_pv(t, sv, true, 1);
@@ -570,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_ref = m_tile;
       }
       const bool rescale_o = li > 0 && __any_sync(0xffffffffu, raise);
-      if (kPHalves == 2 && rescale_o) rescale_o_rows(tO, alpha);
+      if (kPH == 2 && rescale_o) rescale_o_rows(tO, alpha);
       const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
       const float2 sl2v = make_float2(sl2, sl2);
       const float2 nm2 = make_float2(neg_m, neg_m);
@@ -578,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // p = 2^(s * scale * log2 e - m) (the last kEmuPer32 columns of every
       // 32 on the FMA pipe, the rest on MUFU), written as bf16 pairs over the
       // first BN/2 columns of S_t in halves of 64 keys, published on
-      // p_half[2t] (whole tile) or, with kPHalves == 2, each half on its own
+      // p_half[2t] (whole tile) or, with kPH == 2, each half on its own
       // barrier p_half[2t+h] as soon as it is in TMEM.
 #pragma unroll
       for (int h = 0; h < BN / 64; ++h) {
@@ -605,11 +606,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st32(tS + h * 32, pk);
         // whole-P: the rescale waits until the scores have left the registers
-        if (kPHalves == 1 && h == kLastH && rescale_o) rescale_o_rows(tO, alpha);
-        if (kPHalves == 2 || h == kLastH) {
+        if (kPH == 1 && h == kLastH && rescale_o) rescale_o_rows(tO, alpha);
+        if (kPH == 2 || h == kLastH) {
           tmem_wait_st();
           tc_fence_before();
-          uint64_t* pbar = &p_half[2 * t + ((kPHalves == 2 && h == 1) ? 1 : 0)];
+          uint64_t* pbar = &p_half[2 * t + ((kPH == 2 && h == 1) ? 1 : 0)];
           if (PAIR) {
             // one arrival per warp on the even CTA's barrier, after every
             // lane's stores are complete and fenced
