@@ -671,11 +671,13 @@ def run_sparse_experiment(args, w):
 def run_tile_experiment(args, w):
     """Wall-clock time of the fused forward against tile size and head width.
 
-    Key tiles of 64 and 128 (the query tile is the tensor core's 128 rows),
-    head widths 64 and 128, sequence lengths 1K to 64K with the token count
-    B*H*N fixed at 2^19 (so every point holds the same inputs), both masks.
-    One JSON line per point (CUDA-event time per launch, TFLOP/s), then one
-    line per (d, N, mask) naming the faster tile.  Inputs are N(0, 1), seeded.
+    Tile shapes: 256 or 128 query rows per CTA (two 128-row tiles that
+    ping-pong, or one; the query tile is the tensor core's 128 rows) times 128
+    or 64 keys per score tile.  Head widths 64 and 128, sequence lengths 1K to
+    64K with the token count B*H*N fixed at 2^19 (so every point holds the same
+    inputs), both masks.  One JSON line per point (CUDA-event time per launch,
+    TFLOP/s), then one line per (d, N, mask) naming the fastest shape.  Inputs
+    are N(0, 1), seeded.
     """
     import torch
 
@@ -689,6 +691,7 @@ def run_tile_experiment(args, w):
     steps, warmup = max(3, min(args.steps, 20)), args.warmup
     tokens = 1 << 19
     peak, peak_src = tensor_peak()
+    shapes = [(256, 128), (256, 64), (128, 128), (128, 64)]  # (query rows per CTA, keys per tile)
     for d in (64, 128):
         for N in (1024, 4096, 16384, 65536):
             H = tokens // N
@@ -699,21 +702,23 @@ def run_tile_experiment(args, w):
             for causal in (False, True):
                 flops = 4.0 * H * N * N * d / (2 if causal else 1)
                 best = None
-                for key_tile in (64, 128):
-                    ms = time_launches(lambda: fa.fa_fwd_key_tile(q, k, v, o, lse, key_tile=key_tile,
-                                                                  causal=causal, stream=stream),
+                for query_rows, key_tile in shapes:
+                    ms = time_launches(lambda: fa.fa_fwd_tile_config(q, k, v, o, lse, query_rows=query_rows,
+                                                                     key_tile=key_tile, causal=causal,
+                                                                     stream=stream),
                                        steps, warmup, stream)
                     if fa.device_status(stream) != 0:
                         raise RuntimeError("kernel reported a device failure")
                     tf = flops / ms / 1e9
                     pt = {"experiment": "tile_sweep", "B": 1, "H": H, "N": N, "d": d, "causal": causal,
-                          "query_tile": 128, "key_tile": key_tile, "ms": ms, "tflops": tf,
-                          "pct_of_peak": 100.0 * tf / peak, "peak_source": peak_src}
+                          "query_tile": 128, "query_rows_per_cta": query_rows, "key_tile": key_tile,
+                          "ms": ms, "tflops": tf, "pct_of_peak": 100.0 * tf / peak, "peak_source": peak_src}
                     print(json.dumps(pt), flush=True)
-                    if best is None or ms < best[1]:
-                        best = (key_tile, ms)
+                    if best is None or ms < best[2]:
+                        best = (query_rows, key_tile, ms)
                 print(json.dumps({"experiment": "tile_sweep", "summary": True, "N": N, "d": d,
-                                  "causal": causal, "best_key_tile": best[0]}), flush=True)
+                                  "causal": causal, "best_query_rows_per_cta": best[0],
+                                  "best_key_tile": best[1]}), flush=True)
             del q, k, v, o, lse
     return 0
 

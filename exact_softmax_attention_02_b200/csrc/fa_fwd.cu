@@ -162,7 +162,7 @@ struct Cfg {
 // B and loads half of every K/V tile.  Each CTA's TMA signals a local barrier;
 // a forwarding warp then arrives on the even CTA's barrier, so that both CTAs
 // can drain their own copies exactly if they have to unwind.
-template <int D, bool CAUSAL, bool PAIR, bool SPLIT, bool SPARSE, int BN>
+template <int D, bool CAUSAL, bool PAIR, bool SPLIT, bool SPARSE, int BN, int QT>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -172,6 +172,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int QB = C::kQBytes;
   static_assert(BN == BN || !(SPLIT || SPARSE), "split-KV and block-sparse use 128-key tiles");
   constexpr int kPH = BN == 128 ? kPHalves : 1;  // P publications per tile
+  // QT = query tiles per CTA: 2 (the two tiles ping-pong), or 1 for the
+  // tile-size sweep (tile slot 0 stays empty, slot 1 holds the CTA's rows)
+  static_assert(QT == 2 || (QT == 1 && !PAIR && !SPLIT && !SPARSE), "one query tile per CTA: plain forward only");
   constexpr int SB = C::kStageBytes;
   static_assert(!PAIR || D == 128, "the pair kernel splits d = 128 into two 64-wide halves");
   static_assert(!(PAIR && SPLIT), "split-KV uses the single-CTA shape");
@@ -218,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int grp_heads = min(p.group_heads, p.BH - grp * p.group_heads);
   const int bh = grp * p.group_heads + rem % grp_heads;
   const int qblk = p.n_qblk - 1 - rem / grp_heads;
-  const int q0 = qblk * kQTiles * C::kRowsPerTile;  // first row of the block
+  const int q0 = qblk * QT * C::kRowsPerTile - (2 - QT) * C::kRowsPerTile;  // first row of slot 0
   // last key tile each query tile needs (the causal diagonal, or the end)
   int j_last[2];
 #pragma unroll
@@ -256,6 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     n_iter = n;
     first_it[0] = skip;
   }
+  if (QT == 1) first_it[0] = n_iter;  // slot 0 unused
   const bool tile_active[2] = {first_it[0] < n_iter, n_iter > 0};
   // key tile of iteration it
   auto kv_tile = [&](int it) { return SPARSE ? __ldg(blk + n_iter - 1 - it) : kv_end - 1 - it; };
@@ -473,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(mma_done);
       mbar_wait_drain<PAIR>(mma_done, 0, tmo);
     }
-  } else if (warp >= kSoftmaxWarp0) {
+  } else if (warp >= kSoftmaxWarp0 && (QT == 2 || warp >= kSoftmaxWarp0 + 4)) {
     // ------------------------------------------------------------ softmax
     const int t = (warp - kSoftmaxWarp0) >> 2;  // query tile of this warpgroup
     const int wq = warp & 3;                    // TMEM lane quarter
@@ -787,7 +791,7 @@ using host::overlaps;
 struct DeviceInfo {
   bool checked = false;
   bool sm100 = false;
-  bool attr_set[64] = {};
+  bool attr_set[128] = {};
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_devices[kMaxDevices];
@@ -804,7 +808,7 @@ template <int D>
 constexpr bool kUsePair = false;
 #endif
 
-template <int D, bool CAUSAL, bool SPLIT, bool SPARSE = false, int BN = kBN>
+template <int D, bool CAUSAL, bool SPLIT, bool SPARSE = false, int BN = kBN, int QT = kQTiles>
 fa_status launch(const void* Q, const void* K, const void* V, void* O, FwdParams prm, int N, int BH,
                  cudaStream_t stream, DeviceInfo& dev) {
   constexpr bool PAIR = kUsePair<D> && !SPLIT && !SPARSE && BN == kBN;
@@ -816,14 +820,14 @@ fa_status launch(const void* Q, const void* K, const void* V, void* O, FwdParams
     snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed");
     return FA_ERR_CUDA;
   }
-  const long long rows_per_block = static_cast<long long>(kQTiles) * C::kRowsPerTile;
+  const long long rows_per_block = static_cast<long long>(QT) * C::kRowsPerTile;
   prm.n_qblk = static_cast<int>((N + rows_per_block - 1) / rows_per_block);
   const long long units = static_cast<long long>(BH) * prm.n_qblk;
   const long long grid = units * (SPLIT ? prm.num_splits : (PAIR ? 2 : 1));
   if (grid > 0x7fffffffll) return FA_ERR_SHAPE;
-  constexpr int slot = (BN == 64 ? 32 : 0) + (SPARSE ? 16 : 0) + (D == 128 ? 8 : 0) + (CAUSAL ? 4 : 0) +
-                       (PAIR ? 2 : 0) + (SPLIT ? 1 : 0);
-  auto kern = fa_fwd_kernel<D, CAUSAL, PAIR, SPLIT, SPARSE, BN>;
+  constexpr int slot = (QT == 1 ? 64 : 0) + (BN == 64 ? 32 : 0) + (SPARSE ? 16 : 0) + (D == 128 ? 8 : 0) +
+                       (CAUSAL ? 4 : 0) + (PAIR ? 2 : 0) + (SPLIT ? 1 : 0);
+  auto kern = fa_fwd_kernel<D, CAUSAL, PAIR, SPLIT, SPARSE, BN, QT>;
   if (!dev.attr_set[slot]) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -1014,25 +1018,44 @@ fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
                 : launch<64, false, false>(Q, K, V, O, prm, N, bh, st, *dev);
 }
 
-fa_status fa_fwd_key_tile(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
-                          int H, int N, int d, float scale, int causal, int key_tile, void* stream) {
+fa_status fa_fwd_tile_config(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                             int H, int N, int d, float scale, int causal, int query_rows, int key_tile,
+                             void* stream) {
   using namespace fa;
-  if (key_tile == 0 || key_tile == kBN) return fa_fwd(Q, K, V, O, LSE, B, H, N, d, scale, causal, stream);
+  if (query_rows == 0) query_rows = kQTiles * kBM;
+  if (key_tile == 0) key_tile = kBN;
+  if (query_rows == kQTiles * kBM && key_tile == kBN)
+    return fa_fwd(Q, K, V, O, LSE, B, H, N, d, scale, causal, stream);
   FwdParams prm;
   DeviceInfo* dev = nullptr;
   fa_status st0 = check_args(Q, K, V, O, LSE, B, H, N, d, scale);
   if (st0 != FA_OK) return st0;
-  if (key_tile != 64) return FA_ERR_UNSUPPORTED;
+  if ((query_rows != 128 && query_rows != 256) || (key_tile != 64 && key_tile != 128)) return FA_ERR_UNSUPPORTED;
   st0 = prepare(LSE, B, H, N, d, scale, &prm, &dev);
   if (st0 != FA_OK) return st0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int bh = prm.BH;
   std::lock_guard<std::mutex> lock(g_dev_mutex);
+  // (query rows, key tile) in {(256, 64), (128, 128), (128, 64)}; (256, 128) is fa_fwd
+  if (query_rows == 256) {
+    if (d == 128)
+      return causal ? launch<128, true, false, false, 64, 2>(Q, K, V, O, prm, N, bh, st, *dev)
+                    : launch<128, false, false, false, 64, 2>(Q, K, V, O, prm, N, bh, st, *dev);
+    return causal ? launch<64, true, false, false, 64, 2>(Q, K, V, O, prm, N, bh, st, *dev)
+                  : launch<64, false, false, false, 64, 2>(Q, K, V, O, prm, N, bh, st, *dev);
+  }
+  if (key_tile == 128) {
+    if (d == 128)
+      return causal ? launch<128, true, false, false, 128, 1>(Q, K, V, O, prm, N, bh, st, *dev)
+                    : launch<128, false, false, false, 128, 1>(Q, K, V, O, prm, N, bh, st, *dev);
+    return causal ? launch<64, true, false, false, 128, 1>(Q, K, V, O, prm, N, bh, st, *dev)
+                  : launch<64, false, false, false, 128, 1>(Q, K, V, O, prm, N, bh, st, *dev);
+  }
   if (d == 128)
-    return causal ? launch<128, true, false, false, 64>(Q, K, V, O, prm, N, bh, st, *dev)
-                  : launch<128, false, false, false, 64>(Q, K, V, O, prm, N, bh, st, *dev);
-  return causal ? launch<64, true, false, false, 64>(Q, K, V, O, prm, N, bh, st, *dev)
-                : launch<64, false, false, false, 64>(Q, K, V, O, prm, N, bh, st, *dev);
+    return causal ? launch<128, true, false, false, 64, 1>(Q, K, V, O, prm, N, bh, st, *dev)
+                  : launch<128, false, false, false, 64, 1>(Q, K, V, O, prm, N, bh, st, *dev);
+  return causal ? launch<64, true, false, false, 64, 1>(Q, K, V, O, prm, N, bh, st, *dev)
+                : launch<64, false, false, false, 64, 1>(Q, K, V, O, prm, N, bh, st, *dev);
 }
 
 int fa_fwd_splitkv_default_splits(int B, int H, int N, int d, int causal) {

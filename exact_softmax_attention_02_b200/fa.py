@@ -78,9 +78,9 @@ def _load():
     lib.fa_fwd_block_sparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int,
                                         c_float, c_int, vp]
     lib.fa_fwd_block_sparse.restype = c_int
-    lib.fa_fwd_key_tile.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_float, c_int, c_int,
-                                    vp]
-    lib.fa_fwd_key_tile.restype = c_int
+    lib.fa_fwd_tile_config.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_float, c_int, c_int,
+                                       c_int, vp]
+    lib.fa_fwd_tile_config.restype = c_int
     lib.fa_fwd_host.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_size_t, c_int, c_int, c_int, c_int, c_float,
                                 c_int, c_int, vp]
     lib.fa_fwd_host.restype = c_int
@@ -168,9 +168,10 @@ def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
                           B, H, N, d, float(scale), int(bool(causal)), _stream_handle(stream)))
 
 
-def fa_fwd_key_tile(q, k, v, o, lse=None, key_tile: int = 128, scale: float | None = None,
-                    causal: bool = False, stream=None) -> None:
-    """fa_fwd on 128 x ``key_tile`` score tiles (64 or 128), for the tile-size sweep."""
+def fa_fwd_tile_config(q, k, v, o, lse=None, query_rows: int = 256, key_tile: int = 128,
+                       scale: float | None = None, causal: bool = False, stream=None) -> None:
+    """fa_fwd with ``query_rows`` (256 or 128) query rows per CTA and ``key_tile``
+    (128 or 64) keys per score tile, for the tile-size sweep."""
     lib = _load()
     _check_qkvo(q, k, v, o)
     B, H, N, d = q.shape
@@ -179,9 +180,9 @@ def fa_fwd_key_tile(q, k, v, o, lse=None, key_tile: int = 128, scale: float | No
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     with torch.cuda.device(dev):
-        _check(lib.fa_fwd_key_tile(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_ptr,
-                                   B, H, N, d, float(scale), int(bool(causal)), int(key_tile),
-                                   _stream_handle(stream)))
+        _check(lib.fa_fwd_tile_config(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_ptr,
+                                      B, H, N, d, float(scale), int(bool(causal)), int(query_rows),
+                                      int(key_tile), _stream_handle(stream)))
 
 
 def splitkv_workspace_bytes(B: int, H: int, N: int, d: int, num_splits: int = 0,

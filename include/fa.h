@@ -177,18 +177,22 @@ fa_status fa_fwd_splitkv_noalloc(const void* Q, const void* K, const void* V, vo
                                  void* stream);
 
 /*
- * fa_fwd_key_tile -- fa_fwd with a chosen key-tile width, for measuring how
+ * fa_fwd_tile_config -- fa_fwd with a chosen tile shape, for measuring how
  * wall-clock time depends on the tile size (interactiveml.org
  * "FlashAttention saves the matrix, not the quadratic work", the suggested
- * experiments: vary tile size and head width).  key_tile = 128 (or 0) is
- * fa_fwd itself; key_tile = 64 runs the same kernel on 128 x 64 score tiles
- * (twice the key tiles, each half as wide, with a ring of twice as many
- * stages).  The query tile stays 128 rows: the tensor core's M.  Results
- * agree with fa_fwd to rounding.  Arguments and errors as fa_fwd, plus
- * FA_ERR_UNSUPPORTED for any other key_tile.
+ * experiments: vary tile size and head width).
+ *   query_rows  query rows per CTA: 256 (two 128-row tiles whose softmax and
+ *               MMAs ping-pong, as fa_fwd) or 128 (one tile, no ping-pong);
+ *               0 = 256.
+ *   key_tile    keys per score tile: 128 (as fa_fwd) or 64; 0 = 128.
+ * The query tile itself is always 128 rows: the tensor core's M.  (256, 128)
+ * is fa_fwd; the other shapes run the same kernel template and agree with it
+ * to rounding.  Arguments and errors as fa_fwd, plus FA_ERR_UNSUPPORTED for
+ * any other shape.
  */
-fa_status fa_fwd_key_tile(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
-                          int H, int N, int d, float scale, int causal, int key_tile, void* stream);
+fa_status fa_fwd_tile_config(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                             int H, int N, int d, float scale, int causal, int query_rows, int key_tile,
+                             void* stream);
 
 /*
  * fa_fwd_host -- fa_fwd on inputs and outputs in HOST memory: the end-to-end

@@ -208,20 +208,22 @@ def test_block_sparse_argument_checks(lib):
     assert lib.fa_status_string(FA_ERR_LAYOUT).decode().startswith("FA_ERR_LAYOUT")
 
 
-def test_key_tile_argument_checks(lib):
+def test_tile_config_argument_checks(lib):
     vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
-    lib.fa_fwd_key_tile.argtypes = [vp] * 5 + [ci] * 4 + [cf, ci, ci, vp]
-    lib.fa_fwd_key_tile.restype = ci
+    lib.fa_fwd_tile_config.argtypes = [vp] * 5 + [ci] * 4 + [cf, ci, ci, ci, vp]
+    lib.fa_fwd_tile_config.restype = ci
 
-    def kt(key_tile, q=A, d=64):
-        return lib.fa_fwd_key_tile(q, A + 64 * MB, A + 128 * MB, A + 192 * MB, A + 256 * MB,
-                                   1, 1, 1024, d, 0.125, 0, key_tile, None)
+    def tc(query_rows, key_tile, q=A, d=64):
+        return lib.fa_fwd_tile_config(q, A + 64 * MB, A + 128 * MB, A + 192 * MB, A + 256 * MB,
+                                      1, 1, 1024, d, 0.125, 0, query_rows, key_tile, None)
 
-    assert kt(96) == FA_ERR_UNSUPPORTED
-    assert kt(256) == FA_ERR_UNSUPPORTED
-    assert kt(64, q=None) == FA_ERR_NULL
-    assert kt(64, d=32) == FA_ERR_UNSUPPORTED
-    assert kt(128, q=A + 8) == FA_ERR_ALIGN
+    assert tc(256, 96) == FA_ERR_UNSUPPORTED
+    assert tc(256, 256) == FA_ERR_UNSUPPORTED
+    assert tc(64, 128) == FA_ERR_UNSUPPORTED
+    assert tc(512, 64) == FA_ERR_UNSUPPORTED
+    assert tc(128, 64, q=None) == FA_ERR_NULL
+    assert tc(128, 128, d=32) == FA_ERR_UNSUPPORTED
+    assert tc(0, 0, q=A + 8) == FA_ERR_ALIGN
 
 
 def test_host_forward_argument_checks(lib):
