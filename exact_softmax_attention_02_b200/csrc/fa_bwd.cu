@@ -111,15 +111,24 @@ __device__ __forceinline__ void tile_of(const BwdParams& p, bool heavy_high, int
   *tile = heavy_high ? p.n_tiles - 1 - k : k;
 }
 
-// Elementwise step on 16 columns c0..c0+15 of the calling thread's row, on
-// scores s and dp already in registers: p = 2^(s * scale log2e - lse2), 0
-// where `allowed` fails (MASK only); ds = p * (dp - D).  col(c, l4, d4) gives
-// lse2 and D of columns c..c+3.  P (optional) and dS are written back as 8
-// columns of bf16 pairs at c0.
-template <bool WRITE_P, bool MASK, typename Col, typename Allowed>
-__device__ __forceinline__ void p_ds_16(const uint32_t (&s)[16], const uint32_t (&dp)[16], uint32_t tS,
-                                        uint32_t tDP, int c0, float sl2, Col col, Allowed allowed) {
-  uint32_t pk[8], dk[8];
+// tcgen05.wait::ld naming one 16-register destination of the loads it waits
+// for, so that no use of it can be scheduled before the wait.
+__device__ __forceinline__ void tmem_wait_ld_reg16(uint32_t (&a)[16]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7]),
+        "+r"(a[8]), "+r"(a[9]), "+r"(a[10]), "+r"(a[11]), "+r"(a[12]), "+r"(a[13]), "+r"(a[14]),
+        "+r"(a[15])
+      :
+      : "memory");
+}
+
+// Exponentials of 16 columns c0..c0+15 of the calling thread's row, from
+// scores s in registers: p = 2^(s * scale log2e - lse2), 0 where `allowed`
+// fails (MASK only).  col(c, l4, d4) gives lse2 and D of columns c..c+3.
+template <bool MASK, typename Col, typename Allowed>
+__device__ __forceinline__ void p_16(const uint32_t (&s)[16], int c0, float sl2, Col col, Allowed allowed,
+                                     float (&p)[16]) {
   const float2 sl2v = make_float2(sl2, sl2);
 #pragma unroll
   for (int e = 0; e < 16; e += 4) {
@@ -129,47 +138,74 @@ __device__ __forceinline__ void p_ds_16(const uint32_t (&s)[16], const uint32_t 
     for (int u = 0; u < 4; u += 2) {
       const float2 sv = make_float2(__uint_as_float(s[e + u]), __uint_as_float(s[e + u + 1]));
       const float2 lv = u == 0 ? make_float2(-l4.x, -l4.y) : make_float2(-l4.z, -l4.w);
-      const float2 dv = u == 0 ? make_float2(-d4.x, -d4.y) : make_float2(-d4.z, -d4.w);
       const float2 x = ffma2(sv, sl2v, lv);
-      float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      p[e + u] = ex2_approx(x.x);
+      p[e + u + 1] = ex2_approx(x.y);
       if (MASK) {
-        if (!allowed(c0 + e + u)) pv.x = 0.f;
-        if (!allowed(c0 + e + u + 1)) pv.y = 0.f;
+        if (!allowed(c0 + e + u)) p[e + u] = 0.f;
+        if (!allowed(c0 + e + u + 1)) p[e + u + 1] = 0.f;
       }
+    }
+  }
+}
+
+// ds = p * (dp - D) for the same 16 columns; P and dS packed to bf16 pairs.
+template <typename Col>
+__device__ __forceinline__ void ds_16(const float (&p)[16], const uint32_t (&dp)[16], int c0, Col col,
+                                      uint32_t (&pk)[8], uint32_t (&dk)[8]) {
+#pragma unroll
+  for (int e = 0; e < 16; e += 4) {
+    float4 l4, d4;
+    col(c0 + e, l4, d4);
+#pragma unroll
+    for (int u = 0; u < 4; u += 2) {
+      const float2 dv = u == 0 ? make_float2(-d4.x, -d4.y) : make_float2(-d4.z, -d4.w);
+      const float2 pv = make_float2(p[e + u], p[e + u + 1]);
       const float2 g = fadd2(make_float2(__uint_as_float(dp[e + u]), __uint_as_float(dp[e + u + 1])), dv);
       const float2 dsv = fmul2(pv, g);
       pk[(e + u) >> 1] = pack_bf16x2(pv.x, pv.y);
       dk[(e + u) >> 1] = pack_bf16x2(dsv.x, dsv.y);
     }
   }
-  if (WRITE_P) tmem_st8(tS + c0, pk);
-  tmem_st8(tDP + c0, dk);
 }
 
 // The calling thread's share of one tile: 16 columns of each quarter
-// (column h*16 of quarters 0..3), quarter by quarter.  The TMEM loads of the
-// next quarter are issued before the current one is computed; after its
-// stores have completed, each quarter is released on ready[q].
-template <bool WRITE_P, bool MASK, typename Col, typename Allowed>
-__device__ __forceinline__ void p_ds_tile(uint32_t tS, uint32_t tDP, int h, float sl2, Col col,
-                                          Allowed allowed, uint64_t* ready) {
-  uint32_t s[2][16], dp[2][16];
+// (column h*16 of quarters 0..3), quarter by quarter.  Only S is needed for
+// the exponentials, so quarter 0's run while the dP product may still be in
+// the tensor core; dp_ready() waits for it (false: give up) before dP is
+// first read.  The scores of the next quarter are loaded while the current
+// one is computed, and its dP while the current stores drain; P (optional)
+// and dS go back as bf16 pairs over the first 8 of each thread's 16 columns,
+// and each quarter is released on ready[q] once its stores have completed.
+template <bool WRITE_P, bool MASK, typename Col, typename Allowed, typename Wait>
+__device__ __forceinline__ bool p_ds_tile(uint32_t tS, uint32_t tDP, int h, float sl2, Col col,
+                                          Allowed allowed, uint64_t* ready, Wait dp_ready) {
+  uint32_t s[2][16], dp[16];
   tmem_ld16(tS + h * 16, s[0]);
-  tmem_ld16(tDP + h * 16, dp[0]);
-  tmem_wait_ld_regs(s[0], dp[0]);
+  tmem_wait_ld_reg16(s[0]);
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int c0 = q * kQuarter + h * 16;
-    if (q < 3) {
-      tmem_ld16(tS + c0 + kQuarter, s[(q + 1) & 1]);
-      tmem_ld16(tDP + c0 + kQuarter, dp[(q + 1) & 1]);
+    if (q < 3) tmem_ld16(tS + c0 + kQuarter, s[(q + 1) & 1]);
+    float pv[16];
+    p_16<MASK>(s[q & 1], c0, sl2, col, allowed, pv);
+    if (q == 0) {
+      if (!dp_ready()) return false;
+      tc_fence_after();
+      tmem_ld16(tDP + c0, dp);
+      tmem_wait_ld_regs(dp, s[1]);
     }
-    p_ds_16<WRITE_P, MASK>(s[q & 1], dp[q & 1], tS, tDP, c0, sl2, col, allowed);
+    uint32_t pk[8], dk[8];
+    ds_16(pv, dp, c0, col, pk, dk);
+    if (q < 3) tmem_ld16(tDP + c0 + kQuarter, dp);
+    if (WRITE_P) tmem_st8(tS + c0, pk);
+    tmem_st8(tDP + c0, dk);
     tmem_wait_st();
     tc_fence_before();
     mbar_arrive(&ready[q]);
-    if (q < 3) tmem_wait_ld_regs(s[(q + 1) & 1], dp[(q + 1) & 1]);
+    if (q < 3) tmem_wait_ld_regs(dp, s[(q + 1) & 1]);
   }
+  return true;
 }
 
 // Store 32-column chunks [cb, ce) of a 128 x D tile held in TMEM (this
@@ -248,7 +284,7 @@ struct DkdvCfg {
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kSmemTiles = 2 * kTileBytes + kStages * kStageBytes;  // K, V, ring
   static constexpr int kLdBytes = kStages * 2 * kTile * 4;
-  static constexpr int kNumBars = 1 + 2 * kStages + 1 + 4 + 1 + 1;
+  static constexpr int kNumBars = 1 + 2 * kStages + 2 + 4 + 1 + 1;
   static constexpr int kSmemBytes = kSmemTiles + kLdBytes + kNumBars * 8 + 16 + 1024;
 };
 
@@ -278,8 +314,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* kv_full = bars;           // K, V landed
   uint64_t* st_full = bars + 1;       // [S] Q_i, dO_i, LSE2_i, D_i landed
   uint64_t* st_empty = st_full + S;   // [S] MMA done with a stage
-  uint64_t* s_full = st_empty + S;    // S^T and dP^T in TMEM
-  uint64_t* ds_ready = s_full + 1;    // [4] quarter q of P^T and dS^T in TMEM (256 arrivals)
+  uint64_t* s_full = st_empty + S;    // S^T in TMEM
+  uint64_t* dp_full = s_full + 1;     // dP^T in TMEM
+  uint64_t* ds_ready = dp_full + 1;   // [4] quarter q of P^T and dS^T in TMEM (256 arrivals)
   uint64_t* acc_done = ds_ready + 4;  // dK, dV final
   uint64_t* mma_done = acc_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -300,6 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&st_empty[s], 1);
     }
     mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
     for (int q = 0; q < 4; ++q) mbar_init(&ds_ready[q], kElemThreads);
     mbar_init(acc_done, 1);
     mbar_init(mma_done, 1);
@@ -382,8 +420,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t q = sr + s * C::kStageBytes, dO = q + TB;
         issue_abt(tmem + kColS, sk, q);   // S^T = K Q^T
-        issue_abt(tmem + kColDP, sv, dO); // dP^T = V dO^T
         mma_commit(s_full);
+        issue_abt(tmem + kColDP, sv, dO); // dP^T = V dO^T
+        mma_commit(dp_full);
         BWD_TRACE(0, 0, it, 1);
         for (int qq = 0; qq < 4 && ok; ++qq) {
           if (!(ok = mbar_wait(&ds_ready[qq], static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteDs)))
@@ -432,10 +471,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int q0 = i * kTile;
       auto allowed = [&](int c) { return q0 + c >= key; };
       const bool diag = CAUSAL && i == j;
-      if (diag)
-        p_ds_tile<true, true>(tS, tDP, h, sl2, col, allowed, ds_ready);
-      else
-        p_ds_tile<true, false>(tS, tDP, h, sl2, col, allowed, ds_ready);
+      auto dp_ready = [&]() {
+        return __all_sync(0xffffffffu, mbar_wait(dp_full, static_cast<uint32_t>(it) & 1u, abort_flag, status,
+                                                 tmo, kSiteS));
+      };
+      ok = diag ? p_ds_tile<true, true>(tS, tDP, h, sl2, col, allowed, ds_ready, dp_ready)
+                : p_ds_tile<true, false>(tS, tDP, h, sl2, col, allowed, ds_ready, dp_ready);
       if (tr) BWD_TRACE(0, 1 + h, it, 1);
     }
     if (ok) ok = mbar_wait(acc_done, 0, abort_flag, status, tmo, kSiteO);
@@ -480,7 +521,7 @@ struct DqCfg {
   static constexpr int kStages = D == 128 ? 2 : 4;  // each stage: K_j and V_j
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kSmemTiles = 2 * kTileBytes + kStages * kStageBytes;  // Q, dO, ring
-  static constexpr int kNumBars = 1 + 2 * kStages + 1 + 4 + 1 + 1;
+  static constexpr int kNumBars = 1 + 2 * kStages + 2 + 4 + 1 + 1;
   static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 1024;
 };
 
@@ -504,8 +545,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* q_full = bars;
   uint64_t* st_full = bars + 1;
   uint64_t* st_empty = st_full + S;
-  uint64_t* s_full = st_empty + S;
-  uint64_t* ds_ready = s_full + 1;    // [4]
+  uint64_t* s_full = st_empty + S;   // S in TMEM
+  uint64_t* dp_full = s_full + 1;    // dP in TMEM
+  uint64_t* ds_ready = dp_full + 1;  // [4]
   uint64_t* acc_done = ds_ready + 4;
   uint64_t* mma_done = acc_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -525,6 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&st_empty[s], 1);
     }
     mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
     for (int q = 0; q < 4; ++q) mbar_init(&ds_ready[q], kElemThreads);
     mbar_init(acc_done, 1);
     mbar_init(mma_done, 1);
@@ -591,8 +634,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t k = sr + s * C::kStageBytes, v = k + TB;
         issue_abt(tmem + kColS, sq, k);    // S = Q K^T
-        issue_abt(tmem + kColDP, sdo, v);  // dP = dO V^T
         mma_commit(s_full);
+        issue_abt(tmem + kColDP, sdo, v);  // dP = dO V^T
+        mma_commit(dp_full);
         BWD_TRACE(1, 0, it, 1);
         for (int qq = 0; qq < 4 && ok; ++qq) {
           if (!(ok = mbar_wait(&ds_ready[qq], static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteDs)))
@@ -646,10 +690,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int k0 = it * kTile;
       auto allowed = [&](int c) { return k0 + c <= row; };
       const bool diag = CAUSAL && it == i;
-      if (diag)
-        p_ds_tile<false, true>(tS, tDP, h, sl2, col, allowed, ds_ready);
-      else
-        p_ds_tile<false, false>(tS, tDP, h, sl2, col, allowed, ds_ready);
+      auto dp_ready = [&]() {
+        return __all_sync(0xffffffffu, mbar_wait(dp_full, static_cast<uint32_t>(it) & 1u, abort_flag, status,
+                                                 tmo, kSiteS));
+      };
+      ok = diag ? p_ds_tile<false, true>(tS, tDP, h, sl2, col, allowed, ds_ready, dp_ready)
+                : p_ds_tile<false, false>(tS, tDP, h, sl2, col, allowed, ds_ready, dp_ready);
       if (tr) BWD_TRACE(1, 1 + h, it, 1);
     }
     if (ok) ok = mbar_wait(acc_done, 0, abort_flag, status, tmo, kSiteO);
