@@ -521,12 +521,20 @@ struct DqCfg {
   static constexpr int kStages = D == 128 ? 2 : 4;  // each stage: K_j and V_j
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kSmemTiles = 2 * kTileBytes + kStages * kStageBytes;  // Q, dO, ring
-  static constexpr int kNumBars = 1 + 2 * kStages + 2 + 4 + 1 + 1;
+  static constexpr int kNumBars = 1 + 2 * kStages + 2 + 4 + 1 + 1 + 1;
   static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 1024;
+  // Q and dO stay in TMEM for the whole CTA, as the A operands of S and dP
+  // (bf16 pairs, d/2 columns each), next to the dQ accumulator
+  static constexpr uint32_t kColQ = kColAcc + D;
+  static constexpr uint32_t kColDO = kColQ + D / 2;
+  static_assert(kColDO + D / 2 <= kTmemCols, "S, dP, dQ, Q and dO fit in TMEM");
 };
 
 // Same quarter pipeline over the key tiles j: S = Q K_j^T, dP = dO V_j^T, dS
-// in place a quarter (32 keys) at a time, dQ += dS K_j per quarter.
+// in place a quarter (32 keys) at a time, dQ += dS K_j per quarter.  Q and
+// dO are copied once into TMEM, so that S and dP are TS products whose only
+// shared-memory operand is the streamed K or V tile (half the operand reads
+// of an SS product).
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -550,7 +558,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* ds_ready = dp_full + 1;  // [4]
   uint64_t* acc_done = ds_ready + 4;
   uint64_t* mma_done = acc_done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* qt_ready = mma_done + 1;  // Q and dO copied into TMEM (256 arrivals)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qt_ready + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* status = &g_bwd_status;
   const uint64_t tmo = p.timeout_ns;
@@ -571,6 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int q = 0; q < 4; ++q) mbar_init(&ds_ready[q], kElemThreads);
     mbar_init(acc_done, 1);
     mbar_init(mma_done, 1);
+    mbar_init(qt_ready, kElemThreads);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -616,16 +626,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(kTile, kTile, false);
       constexpr uint32_t idAcc = idesc_bf16_f32(kTile, D, true);
-      const uint32_t sq = smem_addr(sQ), sdo = smem_addr(sdO), sr = smem_addr(sRing);
-      auto issue_abt = [&](uint32_t d_tmem, uint32_t a, uint32_t b) {
+      const uint32_t sr = smem_addr(sRing);
+      // X = A B^T with A (Q or dO, 128 rows) in TMEM, B (K or V, 128 rows) K-major in SMEM
+      auto issue_tbt = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-          mma_ss(d_tmem, sw128_desc(a + off, 16, 1024), sw128_desc(b + off, 16, 1024), idS,
-                 kk > 0 ? 1u : 0u);
+          mma_ts(d_tmem, a_tmem + kk * 8, sw128_desc(b + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(q_full, 0, abort_flag, status, tmo, kSiteLoad);
+      bool ok = mbar_wait(qt_ready, 0, abort_flag, status, tmo, kSiteLoad);
       for (int it = 0; it < n_iter && ok; ++it) {
         const int s = it % S;
         if (!(ok = mbar_wait(&st_full[s], static_cast<uint32_t>(it / S) & 1u, abort_flag, status, tmo, kSiteLoad)))
@@ -633,9 +643,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         BWD_TRACE(1, 0, it, 0);
         tc_fence_after();
         const uint32_t k = sr + s * C::kStageBytes, v = k + TB;
-        issue_abt(tmem + kColS, sq, k);    // S = Q K^T
+        issue_tbt(tmem + kColS, tmem + C::kColQ, k);    // S = Q K^T
         mma_commit(s_full);
-        issue_abt(tmem + kColDP, sdo, v);  // dP = dO V^T
+        issue_tbt(tmem + kColDP, tmem + C::kColDO, v);  // dP = dO V^T
         mma_commit(dp_full);
         BWD_TRACE(1, 0, it, 1);
         for (int qq = 0; qq < 4 && ok; ++qq) {
@@ -678,7 +688,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       l4 = l4c;
       d4 = d4c;
     };
-    bool ok = true;
+    // this thread's row of Q (h = 0) or dO (h = 1), from its 128-byte-swizzled
+    // tile into TMEM as bf16 pairs in order: the TS products' A layout
+    bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, status, tmo, kSiteLoad));
+    if (ok) {
+      const uint8_t* src = (h == 0 ? sQ : sdO) + r * 128;
+      const uint32_t dst = tmem + lane_base + (h == 0 ? C::kColQ : C::kColDO);
+#pragma unroll
+      for (int c = 0; c < C::kChunks; ++c) {
+        uint32_t w[32];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const uint4 v = *reinterpret_cast<const uint4*>(src + c * kChunkBytes + ((g ^ (r & 7)) * 16));
+          w[4 * g] = v.x;
+          w[4 * g + 1] = v.y;
+          w[4 * g + 2] = v.z;
+          w[4 * g + 3] = v.w;
+        }
+        tmem_st32(dst + c * 32, w);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(qt_ready);
+    }
     for (int it = 0; it < n_iter && ok; ++it) {
       ok = __all_sync(0xffffffffu,
                       mbar_wait(s_full, static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteS));
