@@ -122,7 +122,8 @@ int fa_fwd_splitkv_default_splits(int B, int H, int N, int d, int causal);
  * D = rowsum(dO * O), dQ = scale dS K, dK = scale dS^T Q).
  *
  *   Q, K, V, O, dO  device, bf16 [B][H][N][d], read (O as written by fa_fwd).
- *   LSE             device, fp32 [B][H][N], read (as written by fa_fwd).
+ *   LSE             device, fp32 [B][H][N], read (as written by fa_fwd with the
+ *                   same scale and mask: finite for every row).
  *   dQ, dK, dV      device, bf16 [B][H][N][d], written.
  *   workspace       device, 16-byte aligned, >= fa_bwd_workspace_bytes(B, H,
  *                   N) bytes, overwritten: LSE * log2(e) and D, each fp32
@@ -217,7 +218,8 @@ fa_status fa_fwd_tile_config(const void* Q, const void* K, const void* V, void* 
  *                O and LSE have reached host memory.  Synchronise it before
  *                reading them.
  * The first call on a device creates the library's three streams and its
- * events (no device memory).  Errors: as fa_fwd, plus FA_ERR_WORKSPACE for a
+ * events (no device memory).  Calls from several host threads are enqueued
+ * one at a time; their work shares the three streams.  Errors: as fa_fwd, plus FA_ERR_WORKSPACE for a
  * short workspace and FA_ERR_UNSUPPORTED when a host argument is device or
  * managed memory or the workspace is not device memory.
  */
