@@ -1,11 +1,15 @@
-"""Exact softmax attention forward for B200 (sm_100a).
+"""Exact softmax attention for B200 (sm_100a): forward, split-KV, block-sparse,
+host-buffer and backward paths.
 
 The compute path is the C-ABI library ``libfa.so`` built from ``csrc/``;
 ``fa.py`` is its thin ctypes binding.  Importing this package does not load
 the library; the first call does, and raises if it is missing.
 """
 
-__all__ = ["fa_fwd", "attention_forward", "FAError", "library_path"]
+__all__ = [
+    "fa_fwd", "fa_fwd_splitkv", "fa_fwd_block_sparse", "fa_fwd_tile_config", "fa_fwd_host", "fa_bwd",
+    "attention_forward", "block_layout_to_csr", "device_status", "FAError", "library_path",
+]
 
 
 def __getattr__(name):
