@@ -723,6 +723,65 @@ def run_tile_experiment(args, w):
     return 0
 
 
+def run_library_experiment(args, w):
+    """Context only: the fused forward beside the attention kernels that torch's
+    scaled_dot_product_attention dispatches to on this GPU (the cuDNN backend
+    and the flash backend), on the same device-resident inputs, same scale
+    and mask.  One JSON line per problem and implementation: average CUDA-event
+    time per launch, TFLOP/s (4*B*H*N^2*d, halved for causal) and the largest
+    |difference| of the library's output from ours.  Not a bench line."""
+    import torch
+    import torch.nn.functional as F
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+
+    from exact_softmax_attention_02_b200 import fa
+
+    if not torch.cuda.is_available():
+        raise SystemExit("the experiment needs a CUDA device")
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    steps, warmup = max(3, min(args.steps, 30)), args.warmup
+    peak, peak_src = tensor_peak()
+    problems = [(2, 16, 8192, 128, True), (1, 32, 32768, 128, True), (2, 16, 16384, 128, False),
+                (4, 16, 4096, 64, False), (2, 16, 8192, 64, True)]
+    for B, H, N, d, causal in problems:
+        g = torch.Generator(device=dev).manual_seed(N + d)
+        q, k, v = (torch.randn(B, H, N, d, device=dev, generator=g).to(torch.bfloat16) for _ in range(3))
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+        scale = d ** -0.5
+        flops = 4.0 * B * H * N * N * d / (2 if causal else 1)
+        impls = [("fa_fwd", None), ("torch_sdpa_cudnn", SDPBackend.CUDNN_ATTENTION),
+                 ("torch_sdpa_flash", SDPBackend.FLASH_ATTENTION)]
+        for name, backend in impls:
+            line = {"experiment": "library_context", "B": B, "H": H, "N": N, "d": d, "causal": causal,
+                    "impl": name}
+            try:
+                if backend is None:
+                    ms = time_launches(lambda: fa.fa_fwd(q, k, v, o, lse, scale=scale, causal=causal,
+                                                         stream=stream), steps, warmup, stream)
+                    if fa.device_status(stream) != 0:
+                        raise RuntimeError("kernel reported a device failure")
+                else:
+                    with sdpa_kernel(backend):
+                        ref = F.scaled_dot_product_attention(q, k, v, is_causal=causal, scale=scale)
+                        line["max_abs_diff_vs_fa_fwd"] = (ref.float() - o.float()).abs().max().item()
+                        del ref
+                        ms = time_launches(lambda: F.scaled_dot_product_attention(q, k, v, is_causal=causal,
+                                                                                  scale=scale),
+                                           steps, warmup, stream)
+            except RuntimeError as e:  # a backend this torch build cannot run here
+                line["unavailable"] = str(e).splitlines()[0][:160]
+                print(json.dumps(line), flush=True)
+                continue
+            tf = flops / ms / 1e9
+            line.update({"ms": ms, "tflops": tf, "pct_of_peak": 100.0 * tf / peak, "peak_source": peak_src})
+            print(json.dumps(line), flush=True)
+        del q, k, v, o, lse
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main(argv=None):
     from exact_softmax_attention_02_b200.inputs import WORKLOADS
 
@@ -737,10 +796,11 @@ def main(argv=None):
                          "standard: the materialising comparator (GEMM, softmax, GEMM); "
                          "backward: fa_bwd (dQ, dK, dV)")
     ap.add_argument("--splits", type=int, default=0, help="splitkv: key ranges (0 = default)")
-    ap.add_argument("--experiment", default=None, choices=["sparse", "tiles"],
+    ap.add_argument("--experiment", default=None, choices=["sparse", "tiles", "library"],
                     help="sparse: exact vs block-sparse bands at matched output error; tiles: "
-                         "time against key-tile width and head width (1 GPU, JSON lines; not a "
-                         "bench line)")
+                         "time against key-tile width and head width; library: the fused forward "
+                         "beside torch's cuDNN and flash attention kernels, for context (1 GPU, "
+                         "JSON lines; not a bench line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-step-seconds", type=float, default=8.0,
                     help="reference arm: target oracle seconds per step (bounded sample)")
@@ -763,6 +823,8 @@ def main(argv=None):
         return run_sparse_experiment(args, w)
     if args.experiment == "tiles":
         return run_tile_experiment(args, w)
+    if args.experiment == "library":
+        return run_library_experiment(args, w)
     return run_ours(args, w)
 
 
