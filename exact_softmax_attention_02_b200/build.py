@@ -1,6 +1,6 @@
 """Build libfa.so in-tree with nvcc for sm_100a.
 
-    python -m exact_softmax_attention_02_b200.build [--force] [--verbose]
+    python -m exact_softmax_attention_02_b200.build [--force] [--verbose] [--trace]
 
 The library is built from csrc/fa_fwd.cu (the fused forward, split-KV,
 merge, block-sparse and key-tile variants), csrc/fa_bwd.cu (the backward
@@ -25,6 +25,9 @@ SOURCES = [os.path.join(HERE, "csrc", n)
 DEPENDS = SOURCES + [os.path.join(HERE, "csrc", "sm100.cuh"), os.path.join(HERE, "csrc", "host_util.h"),
                      os.path.join(ROOT, "include", "fa.h")]
 OUTPUT = os.path.join(HERE, "libfa.so")
+# the same sources built with -DFA_TRACE: SM clock stamps of the forward's
+# phases (phase_trace.py reads them); never loaded unless FA_LIBRARY names it
+TRACE_OUTPUT = os.path.join(HERE, "libfa_trace.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -41,31 +44,34 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(OUTPUT):
+def up_to_date(output: str = OUTPUT) -> bool:
+    if not os.path.exists(output):
         return False
-    t = os.path.getmtime(OUTPUT)
+    t = os.path.getmtime(output)
     return all(os.path.getmtime(p) <= t for p in DEPENDS)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return OUTPUT
-    tmp = OUTPUT + ".tmp"
-    cmd = [nvcc(), *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), "-o", tmp, *SOURCES]
+def build(force: bool = False, verbose: bool = False, trace: bool = False) -> str:
+    output = TRACE_OUTPUT if trace else OUTPUT
+    if not force and up_to_date(output):
+        return output
+    tmp = output + ".tmp"
+    cmd = [nvcc(), *NVCC_FLAGS, *(["-DFA_TRACE"] if trace else []), *(["-Xptxas", "-v"] if verbose else []),
+           "-o", tmp, *SOURCES]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)
         raise RuntimeError("nvcc failed: " + " ".join(cmd))
     if verbose:
         sys.stderr.write(res.stderr)
-    os.replace(tmp, OUTPUT)
-    return OUTPUT
+    os.replace(tmp, output)
+    return output
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--trace", action="store_true", help="build libfa_trace.so (-DFA_TRACE) instead")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose))
+    print(build(force=a.force, verbose=a.verbose, trace=a.trace))
