@@ -315,6 +315,80 @@ def run_reference(args, w):
     return 0
 
 
+# The other configurations the target names, measured in the same run as the
+# headline (one GPU only): the d=64 problem, the two long-context causal
+# problems, and the backward pass of the headline problem.
+EXTRA_CONFIGS = [
+    ("b4h16n4096d64", "forward"),
+    ("b1h32n32768d128_causal_q4", "forward"),
+    ("b1h8n131072d128_causal", "forward"),
+    ("b2h16n8192d128_causal", "backward"),
+]
+
+
+def measure_config(name: str, path: str, dev, steps: int = 20, warmup: int = 5):
+    """Kernel throughput of one more configuration: W untimed launches, then
+    K launches timed with CUDA events on the launching stream, clocks sampled
+    during the timed launches.  Returns a dict for the bench line."""
+    import torch
+
+    from exact_softmax_attention_02_b200 import fa
+    from exact_softmax_attention_02_b200.inputs import WORKLOADS, make_workload_inputs
+
+    w = WORKLOADS[name]
+    q, k, v = (t.to(dev) for t in make_workload_inputs(w))
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flops = w.flops
+    if path == "backward":
+        fa.fa_fwd(q, k, v, o, lse, scale=w.scale, causal=w.causal, stream=stream)
+        g = torch.Generator(device="cpu").manual_seed(w.seed + 100)
+        do = torch.randn(q.shape, generator=g).to(torch.bfloat16).to(dev)
+        grads = [torch.empty_like(q) for _ in range(3)]
+        ws = torch.empty(max(16, fa.bwd_workspace_bytes(w.B, w.H, w.N)), dtype=torch.uint8, device=dev)
+        flops *= 2.5  # five N^2 d products against the forward's two
+
+        def step():
+            fa.fa_bwd(q, k, v, o, do, lse, *grads, workspace=ws, scale=w.scale, causal=w.causal,
+                      stream=stream)
+    else:
+        def step():
+            fa.fa_fwd(q, k, v, o, lse, scale=w.scale, causal=w.causal, stream=stream)
+
+    for _ in range(warmup):
+        step()
+    if fa.device_status(stream) != 0:
+        raise RuntimeError(f"{name} {path}: kernel reported a device failure in warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    sampler = ClockSampler(dev.index, period_s=float(os.environ.get("FA_BENCH_CLOCK_PERIOD", "0.01")))
+    sampler.start()
+    torch.cuda.synchronize(dev)
+    for a, b in ev:
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.stop()
+    if fa.device_status(stream) != 0:
+        raise RuntimeError(f"{name} {path}: kernel reported a device failure")
+    ms = sorted(a.elapsed_time(b) for a, b in ev)
+    mean_s = sum(ms) / len(ms) / 1e3
+    peak, _ = tensor_peak()
+    tf = flops / mean_s / 1e12
+    out = {"path": path, "tflops": tf, "frac": tf / peak, "ms_per_step": 1e3 * mean_s,
+           "ms_min": ms[0], "ms_median": ms[len(ms) // 2], "steps": steps, "warmup": warmup,
+           "flops_per_step": flops, "clocks": sampler.summary(),
+           "kernel": ("bwd_rowdot + bwd_dkdv_kernel + bwd_dq_kernel" if path == "backward"
+                      else f"fa_fwd_kernel<{w.d},{str(w.causal).lower()}>"),
+           "launches": steps * (3 if path == "backward" else 1)}
+    if path == "backward":
+        out["flops_convention"] = "2.5 x forward (five N^2 d products)"
+    del q, k, v, o, lse
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, w):
     import torch
 
@@ -491,6 +565,15 @@ def run_ours(args, w):
     if rank == 0 and world == 1 and not args.no_cpu_baseline and bwd is None:
         cpu = cpu_baseline(w, w.seed)
 
+    # the other configurations of the target, on one GPU only (a multi-GPU
+    # run reports the headline problem alone)
+    per_config = None
+    if world == 1 and not args.no_per_config and args.path == "fused" and w.name == DEFAULT_WORKLOAD:
+        per_config = {}
+        for name, path in EXTRA_CONFIGS:
+            key = name if path == "forward" else f"{name}_backward"
+            per_config[key] = measure_config(name, path, dev)
+
     if dist is not None:
         dist.barrier()
     if rank == 0:
@@ -514,6 +597,7 @@ def run_ours(args, w):
             "step_ms": step_ms,
             "clocks": clocks,
             "cpu_baseline": cpu,
+            **({"per_config": per_config} if per_config is not None else {}),
         }
         print(json.dumps(line), flush=True)
     if dist is not None:
@@ -723,65 +807,6 @@ def run_tile_experiment(args, w):
     return 0
 
 
-def run_library_experiment(args, w):
-    """Context only: the fused forward beside the attention kernels that torch's
-    scaled_dot_product_attention dispatches to on this GPU (the cuDNN backend
-    and the flash backend), on the same device-resident inputs, same scale
-    and mask.  One JSON line per problem and implementation: average CUDA-event
-    time per launch, TFLOP/s (4*B*H*N^2*d, halved for causal) and the largest
-    |difference| of the library's output from ours.  Not a bench line."""
-    import torch
-    import torch.nn.functional as F
-    from torch.nn.attention import SDPBackend, sdpa_kernel
-
-    from exact_softmax_attention_02_b200 import fa
-
-    if not torch.cuda.is_available():
-        raise SystemExit("the experiment needs a CUDA device")
-    dev = torch.device("cuda", 0)
-    stream = torch.cuda.current_stream(dev)
-    steps, warmup = max(3, min(args.steps, 30)), args.warmup
-    peak, peak_src = tensor_peak()
-    problems = [(2, 16, 8192, 128, True), (1, 32, 32768, 128, True), (2, 16, 16384, 128, False),
-                (4, 16, 4096, 64, False), (2, 16, 8192, 64, True)]
-    for B, H, N, d, causal in problems:
-        g = torch.Generator(device=dev).manual_seed(N + d)
-        q, k, v = (torch.randn(B, H, N, d, device=dev, generator=g).to(torch.bfloat16) for _ in range(3))
-        o = torch.empty_like(q)
-        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
-        scale = d ** -0.5
-        flops = 4.0 * B * H * N * N * d / (2 if causal else 1)
-        impls = [("fa_fwd", None), ("torch_sdpa_cudnn", SDPBackend.CUDNN_ATTENTION),
-                 ("torch_sdpa_flash", SDPBackend.FLASH_ATTENTION)]
-        for name, backend in impls:
-            line = {"experiment": "library_context", "B": B, "H": H, "N": N, "d": d, "causal": causal,
-                    "impl": name}
-            try:
-                if backend is None:
-                    ms = time_launches(lambda: fa.fa_fwd(q, k, v, o, lse, scale=scale, causal=causal,
-                                                         stream=stream), steps, warmup, stream)
-                    if fa.device_status(stream) != 0:
-                        raise RuntimeError("kernel reported a device failure")
-                else:
-                    with sdpa_kernel(backend):
-                        ref = F.scaled_dot_product_attention(q, k, v, is_causal=causal, scale=scale)
-                        line["max_abs_diff_vs_fa_fwd"] = (ref.float() - o.float()).abs().max().item()
-                        del ref
-                        ms = time_launches(lambda: F.scaled_dot_product_attention(q, k, v, is_causal=causal,
-                                                                                  scale=scale),
-                                           steps, warmup, stream)
-            except RuntimeError as e:  # a backend this torch build cannot run here
-                line["unavailable"] = str(e).splitlines()[0][:160]
-                print(json.dumps(line), flush=True)
-                continue
-            tf = flops / ms / 1e9
-            line.update({"ms": ms, "tflops": tf, "pct_of_peak": 100.0 * tf / peak, "peak_source": peak_src})
-            print(json.dumps(line), flush=True)
-        del q, k, v, o, lse
-        torch.cuda.empty_cache()
-    return 0
-
-
 def main(argv=None):
     from exact_softmax_attention_02_b200.inputs import WORKLOADS
 
@@ -796,12 +821,14 @@ def main(argv=None):
                          "standard: the materialising comparator (GEMM, softmax, GEMM); "
                          "backward: fa_bwd (dQ, dK, dV)")
     ap.add_argument("--splits", type=int, default=0, help="splitkv: key ranges (0 = default)")
-    ap.add_argument("--experiment", default=None, choices=["sparse", "tiles", "library"],
+    ap.add_argument("--experiment", default=None, choices=["sparse", "tiles"],
                     help="sparse: exact vs block-sparse bands at matched output error; tiles: "
-                         "time against key-tile width and head width; library: the fused forward "
-                         "beside torch's cuDNN and flash attention kernels, for context (1 GPU, "
-                         "JSON lines; not a bench line)")
+                         "time against key-tile width and head width (1 GPU, JSON lines; not a "
+                         "bench line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the other configurations (d=64, long-context causal, backward) "
+                         "measured after the headline problem")
     ap.add_argument("--ref-step-seconds", type=float, default=8.0,
                     help="reference arm: target oracle seconds per step (bounded sample)")
     args = ap.parse_args(argv)
@@ -823,8 +850,6 @@ def main(argv=None):
         return run_sparse_experiment(args, w)
     if args.experiment == "tiles":
         return run_tile_experiment(args, w)
-    if args.experiment == "library":
-        return run_library_experiment(args, w)
     return run_ours(args, w)
 
 

@@ -163,8 +163,8 @@ __device__ __forceinline__ void ds_16(const float (&p)[16], const uint32_t (&dp)
       const float2 pv = make_float2(p[e + u], p[e + u + 1]);
       const float2 g = fadd2(make_float2(__uint_as_float(dp[e + u]), __uint_as_float(dp[e + u + 1])), dv);
       const float2 dsv = fmul2(pv, g);
-      pk[(e + u) >> 1] = pack_bf16x2(pv.x, pv.y);
-      dk[(e + u) >> 1] = pack_bf16x2(dsv.x, dsv.y);
+      pk[(e + u) >> 1] = round_pack_bf16x2(pv.x, pv.y);
+      dk[(e + u) >> 1] = round_pack_bf16x2(dsv.x, dsv.y);
     }
   }
 }
@@ -761,19 +761,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 namespace {
 
-std::mutex g_attr_mutex;
-bool g_attr_set[64][8] = {};
+// dynamic shared-memory attribute set per (device, kernel); the call is
+// idempotent, so threads that race on an unset flag both make it, harmlessly
+std::atomic<bool> g_attr_set[64][8] = {};
 
 template <typename Kern>
 fa_status set_smem(Kern kern, int bytes, int slot) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return host::cuda_fail(e, "cudaGetDevice");
-  std::lock_guard<std::mutex> lock(g_attr_mutex);
-  if (!g_attr_set[dev & 63][slot]) {
+  if (!g_attr_set[dev & 63][slot].load(std::memory_order_acquire)) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return host::cuda_fail(e, "cudaFuncSetAttribute");
-    g_attr_set[dev & 63][slot] = true;
+    g_attr_set[dev & 63][slot].store(true, std::memory_order_release);
   }
   return FA_OK;
 }
@@ -784,10 +784,10 @@ fa_status launch_bwd(const void* Q, const void* K, const void* V, const void* O,
                      cudaStream_t st) {
   const int N = prm.N, BH = prm.BH;
   CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv;
-  if (!host::make_map(&mq, Q, D, N, BH, kTile) || !host::make_map(&mk, K, D, N, BH, kTile) ||
-      !host::make_map(&mv, V, D, N, BH, kTile) || !host::make_map(&mdo, dO, D, N, BH, kTile) ||
-      !host::make_map(&mdq, dQ, D, N, BH, kTile) || !host::make_map(&mdk, dK, D, N, BH, kTile) ||
-      !host::make_map(&mdv, dV, D, N, BH, kTile)) {
+  if (!host::make_map_cached(&mq, Q, D, N, BH, kTile) || !host::make_map_cached(&mk, K, D, N, BH, kTile) ||
+      !host::make_map_cached(&mv, V, D, N, BH, kTile) || !host::make_map_cached(&mdo, dO, D, N, BH, kTile) ||
+      !host::make_map_cached(&mdq, dQ, D, N, BH, kTile) || !host::make_map_cached(&mdk, dK, D, N, BH, kTile) ||
+      !host::make_map_cached(&mdv, dV, D, N, BH, kTile)) {
     snprintf(host::g_last_error, sizeof(host::g_last_error), "cuTensorMapEncodeTiled failed");
     return FA_ERR_CUDA;
   }

@@ -49,6 +49,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "fa.h"
@@ -68,25 +69,11 @@ static_assert(FA_BLOCK_Q == kQTiles * kBM && FA_BLOCK_K == kBN,
 constexpr int kThreads = 384;  // 12 warps
 constexpr int kSoftmaxWarp0 = 4;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-#ifndef FA_EMU_PER32
-#define FA_EMU_PER32 0
-#endif
-// columns (of every 32) whose exponential runs on the FMA pipe instead of MUFU
-constexpr int kEmuPer32 = FA_EMU_PER32;
-static_assert(kEmuPer32 >= 0 && kEmuPer32 <= 32 && kEmuPer32 % 2 == 0, "even count per 32");
-#ifndef FA_P_HALVES
-#define FA_P_HALVES 1
-#endif
-// 1: P_t is published once per tile; 2: in two halves of 64 keys, each on its
-// own barrier, so that the PV product can start on the first half (128-key
-// tiles only; 64-key tiles always publish P whole)
-constexpr int kPHalves = FA_P_HALVES;
-static_assert(kPHalves == 1 || kPHalves == 2, "P is published whole or in two halves");
 constexpr uint32_t kTmemCols = 512;
 // wait sites reported in the device status word (bit 8 + site)
 enum : uint32_t {
-  kSiteKvEmpty = 0, kSiteQ = 1, kSiteKvFull = 2, kSiteS = 3, kSiteP = 4,  // 4..7: p_half[0..3]
-  kSiteO = 8, kSiteDebug = 9, kSiteLand = 10,
+  kSiteKvEmpty = 0, kSiteQ = 1, kSiteKvFull = 2, kSiteS = 3, kSiteP = 4,  // 4..5: p_full[0..1]
+  kSiteO = 8, kSiteDebug = 9,
 };
 constexpr int kChunkBytes = kBM * 64 * 2;  // one 64-wide, 128-row swizzled box: 16 KB
 
@@ -116,6 +103,25 @@ struct FwdParams {
 
 __device__ uint32_t g_device_status;
 
+// Index checks of the debug build (compiled with -DFA_DEBUG): every shared
+// memory, tensor memory and global index the kernels compute at run time is
+// checked before the access it guards.  A failed check raises kStatusBounds
+// and bit 16 + site in the device status word, the access is skipped, and the
+// CTA unwinds as after a wait that gave up; nothing traps.  In the normal
+// build the checks compile to nothing.
+enum : uint32_t {
+  kCheckQLoad = 0, kCheckKvLoad = 1, kCheckLse = 2, kCheckPartial = 3, kCheckStage = 4,
+  kCheckStore = 5, kCheckMerge = 6, kCheckTmem = 7,
+};
+#ifdef FA_DEBUG
+__device__ __forceinline__ bool in_bounds(bool ok, uint32_t site) {
+  if (!ok) atomicOr(&g_device_status, kStatusBounds | (1u << (16 + (site & 15u))));
+  return ok;
+}
+#else
+__device__ __forceinline__ constexpr bool in_bounds(bool, uint32_t) { return true; }
+#endif
+
 // Optional phase trace (build with -DFA_TRACE): SM clock stamps of the MMA
 // issuer and of one thread per softmax warpgroup, for the first CTAs.
 #ifdef FA_TRACE
@@ -134,51 +140,37 @@ __device__ unsigned long long* g_trace;  // [kTraceCtas][4 roles][kTraceIters][8
   } while (0)
 #endif
 
-template <int D, bool PAIR, int BN = kBN>
+template <int D, int BN = kBN>
 struct Cfg {
-  static_assert(BN == 128 || (BN == 64 && !PAIR), "key tiles of 128, or 64 on one CTA");
+  static_assert(BN == 128 || BN == 64, "key tiles of 128 or 64");
   static constexpr int kChunks = D / 64;
   static constexpr int kQBytes = kBM * D * 2;  // one query tile (reused as O staging)
-  // one ring stage: a whole K or V tile, or (PAIR) this CTA's half of one
-  static constexpr int kStageBytes = PAIR ? BN * D : BN * D * 2;
-  static constexpr int kKRows = PAIR ? BN / 2 : BN;  // key rows of a K stage
-  static constexpr int kKChunkBytes = kKRows * 128;  // one 64-wide d chunk of a K stage
-  static constexpr int kVChunkBytes = BN * 128;      // one 64-wide d chunk of a V stage
+  static constexpr int kStageBytes = BN * D * 2;  // one ring stage: a whole K or V tile
+  static constexpr int kKChunkBytes = BN * 128;   // one 64-wide d chunk of a K stage
+  static constexpr int kVChunkBytes = BN * 128;   // one 64-wide d chunk of a V stage
   // the same ring bytes whatever the tile: more stages for smaller tiles
-  static constexpr int kStages = ((PAIR || D == 64) ? 8 : 4) * (128 / BN);
-  static constexpr int kRowsPerTile = PAIR ? 2 * kBM : kBM;  // rows of one (pair) MMA tile
-  static constexpr int kNumBars = 2 + 2 + 3 * kStages + 2 + 4 + 2 + 1 + 1;
+  static constexpr int kStages = (D == 64 ? 8 : 4) * (128 / BN);
+  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 1 + 1;
   static constexpr int kSmemTiles = kQTiles * kQBytes + kStages * kStageBytes;
   static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 1024;
   static constexpr uint32_t kColO = 256;
 };
 
-// One kernel for both CTA shapes.  PAIR == false: one CTA owns two 128-row
-// query tiles and issues M=128 MMAs.  PAIR == true (d = 128): a cluster of
-// two CTAs owns two 256-row tiles; tile t of CTA r is rows 256t + 128r of the
-// pair's 512; the even CTA issues M=256 MMAs whose B operand (K for S, V for
-// PV) is split between the two CTAs' shared memory -- keys 64r..64r+63 of each
-// K tile and d columns 64r..64r+63 of each V tile -- so each CTA reads half of
-// B and loads half of every K/V tile.  Each CTA's TMA signals a local barrier;
-// a forwarding warp then arrives on the even CTA's barrier, so that both CTAs
-// can drain their own copies exactly if they have to unwind.
-template <int D, bool CAUSAL, bool PAIR, bool SPLIT, bool SPARSE, int BN, int QT>
+// One CTA owns two 128-row query tiles of one head and issues M=128 MMAs.
+template <int D, bool CAUSAL, bool SPLIT, bool SPARSE, int BN, int QT>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const FwdParams p) {
-  using C = Cfg<D, PAIR, BN>;
+  using C = Cfg<D, BN>;
   constexpr int S = C::kStages;
   constexpr int QB = C::kQBytes;
-  static_assert(BN == BN || !(SPLIT || SPARSE), "split-KV and block-sparse use 128-key tiles");
-  constexpr int kPH = BN == 128 ? kPHalves : 1;  // P publications per tile
+  static_assert(BN == 128 || !(SPLIT || SPARSE), "split-KV and block-sparse use 128-key tiles");
   // QT = query tiles per CTA: 2 (the two tiles ping-pong), or 1 for the
   // tile-size sweep (tile slot 0 stays empty, slot 1 holds the CTA's rows)
-  static_assert(QT == 2 || (QT == 1 && !PAIR && !SPLIT && !SPARSE), "one query tile per CTA: plain forward only");
+  static_assert(QT == 2 || (QT == 1 && !SPLIT && !SPARSE), "one query tile per CTA: plain forward only");
   constexpr int SB = C::kStageBytes;
-  static_assert(!PAIR || D == 128, "the pair kernel splits d = 128 into two 64-wide halves");
-  static_assert(!(PAIR && SPLIT), "split-KV uses the single-CTA shape");
-  static_assert(!(SPARSE && (PAIR || SPLIT)), "block-sparse uses the single-CTA, unsplit shape");
+  static_assert(!(SPARSE && SPLIT), "block-sparse uses the unsplit shape");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -186,31 +178,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = smem;                  // kQTiles query tiles (reused as O staging)
   uint8_t* sKV = smem + kQTiles * QB;  // S ring stages
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemTiles);
-  uint64_t* q_land = bars;            // [2] own Q copies landed (PAIR; else alias of q_full)
-  uint64_t* q_full = bars + 2;        // [2] Q tile ready for the MMA
-  uint64_t* kv_land = q_full + 2;     // [S] own K/V copies landed (PAIR; else alias of kv_full)
-  uint64_t* kv_full = kv_land + S;    // [S] K/V stage ready for the MMA
-  uint64_t* kv_empty = kv_full + S;   // [S] MMA -> producers
+  uint64_t* q_full = bars;            // [2] Q tile landed
+  uint64_t* kv_full = q_full + 2;     // [S] K/V stage landed
+  uint64_t* kv_empty = kv_full + S;   // [S] MMA -> producer
   uint64_t* s_full = kv_empty + S;    // [2] MMA -> softmax
-  uint64_t* p_half = s_full + 2;      // [4] softmax -> MMA, [2t+h]
-  uint64_t* o_full = p_half + 4;      // [2] MMA -> epilogue
+  uint64_t* p_full = s_full + 2;      // [2] softmax -> MMA
+  uint64_t* o_full = p_full + 2;      // [2] MMA -> epilogue
   uint64_t* mma_done = o_full + 2;    // [1] MMA -> itself, before TMEM release
   uint64_t* never = mma_done + 1;     // [1] debug: nothing arrives here
-  if (!PAIR) {
-    q_land = q_full;
-    kv_land = kv_full;
-  }
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* status = &g_device_status;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
   const int split = SPLIT ? static_cast<int>(blockIdx.x % p.num_splits) : 0;
-  const int unit = SPLIT  ? static_cast<int>(blockIdx.x / p.num_splits)
-                   : PAIR ? static_cast<int>(blockIdx.x >> 1)
-                          : static_cast<int>(blockIdx.x);
+  const int unit = SPLIT ? static_cast<int>(blockIdx.x / p.num_splits) : static_cast<int>(blockIdx.x);
   // Work order: heads in groups of p.group_heads; inside a group, query
   // blocks from the heaviest (last rows: most keys when causal) to the
   // lightest, cycling over the group's heads.  Blocks that run together then
@@ -221,12 +204,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int grp_heads = min(p.group_heads, p.BH - grp * p.group_heads);
   const int bh = grp * p.group_heads + rem % grp_heads;
   const int qblk = p.n_qblk - 1 - rem / grp_heads;
-  const int q0 = qblk * QT * C::kRowsPerTile - (2 - QT) * C::kRowsPerTile;  // first row of slot 0
+  const int q0 = qblk * QT * kBM - (2 - QT) * kBM;  // first row of slot 0
   // last key tile each query tile needs (the causal diagonal, or the end)
   int j_last[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t)
-    j_last[t] = CAUSAL ? min(q0 + (t + 1) * C::kRowsPerTile - 1, p.N - 1) / BN : p.n_kv - 1;
+    j_last[t] = CAUSAL ? min(q0 + (t + 1) * kBM - 1, p.N - 1) / BN : p.n_kv - 1;
   // key tiles [kv_lo, kv_end) of this CTA (all of them unless split), visited
   // from kv_end-1 down to kv_lo
   const int kv_lo = SPLIT ? split * p.kv_per_split : 0;
@@ -267,17 +250,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
-      if (PAIR) mbar_init(&q_land[t], 1);
-      mbar_init(&q_full[t], PAIR ? 2 : 1);
+      mbar_init(&q_full[t], 1);
       mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], kBM);
       mbar_init(&o_full[t], 1);
     }
     for (int s = 0; s < S; ++s) {
-      if (PAIR) mbar_init(&kv_land[s], 1);
-      mbar_init(&kv_full[s], PAIR ? 2 : 1);
+      mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    for (int h = 0; h < 4; ++h) mbar_init(&p_half[h], PAIR ? 2 * (kBM / 32) : kBM);
     mbar_init(mma_done, 1);
     mbar_init(never, 1);
     *abort_flag = 0;
@@ -288,33 +269,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmO);
   }
   if (warp == 1) {
-    if (PAIR) {
-      tmem_alloc_pair(tmem_slot, kTmemCols);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(tmem_slot, kTmemCols);
-      tmem_relinquish();
-    }
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
   }
   tc_fence_before();
-  if (PAIR)
-    cluster_sync();
-  else
-    __syncthreads();
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  static_assert(2 * BN <= C::kColO && C::kColO + 2 * D <= kTmemCols, "S_0, S_1, O_0, O_1 fit the allocation");
+  // (all 512 columns are allocated, so the base column is 0)
+  if (threadIdx.x == 0) in_bounds((tmem & 0xffffu) == 0, kCheckTmem);
 
   // rows of this CTA's query tile t
-  auto tile_row0 = [&](int t) { return q0 + t * C::kRowsPerTile + (PAIR ? static_cast<int>(rank) * kBM : 0); };
+  auto tile_row0 = [&](int t) { return q0 + t * kBM; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && n_iter > 0) {
       bool ok = true;
+      bool q_issued[2] = {false, false};
       if (tile_active[0]) {
-        mbar_arrive_expect_tx(&q_land[0], QB);
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(sQ + c * kChunkBytes, &tmQ, &q_land[0], c * 64, tile_row0(0), bh);
+        if (in_bounds(tile_row0(0) >= 0 && tile_row0(0) < p.N && bh < p.BH, kCheckQLoad)) {
+          q_issued[0] = true;
+          mbar_arrive_expect_tx(&q_full[0], QB);
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d(sQ + c * kChunkBytes, &tmQ, &q_full[0], c * 64, tile_row0(0), bh);
+        } else {
+          ok = false;
+          *abort_flag = 1;
+        }
       }
       int i = 0;  // loads issued into the ring, in consumption order K0 V0 K1 V1 ...
       for (int it = 0; it < n_iter && ok; ++it) {
@@ -323,25 +306,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kv = 0; kv < 2; ++kv) {
           const int s = i % S;
           const uint32_t ph = static_cast<uint32_t>(i / S) & 1u;
-          ok = mbar_wait<PAIR>(&kv_empty[s], ph ^ 1u, abort_flag, status, tmo, kSiteKvEmpty);
+          ok = mbar_wait(&kv_empty[s], ph ^ 1u, abort_flag, status, tmo, kSiteKvEmpty);
           if (!ok) break;
-          mbar_arrive_expect_tx(&kv_land[s], SB);
-          uint8_t* st = sKV + s * SB;
-          if (kv == 0) {
-            for (int c = 0; c < C::kChunks; ++c)
-              tma_load_3d(st + c * C::kKChunkBytes, &tmK, &kv_land[s], c * 64,
-                          j * BN + static_cast<int>(rank) * C::kKRows, bh);
-          } else if (PAIR) {
-            tma_load_3d(st, &tmV, &kv_land[s], static_cast<int>(rank) * 64, j * BN, bh);
-          } else {
-            for (int c = 0; c < C::kChunks; ++c)
-              tma_load_3d(st + c * C::kVChunkBytes, &tmV, &kv_land[s], c * 64, j * BN, bh);
+          if (!in_bounds(j >= 0 && j < p.n_kv && s < S && bh < p.BH, kCheckKvLoad)) {
+            ok = false;
+            *abort_flag = 1;
+            break;
           }
+          mbar_arrive_expect_tx(&kv_full[s], SB);
+          uint8_t* st = sKV + s * SB;
+          const CUtensorMap* map = kv == 0 ? &tmK : &tmV;
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d(st + c * C::kKChunkBytes, map, &kv_full[s], c * 64, j * BN, bh);
           ++i;
           if (it == 0 && kv == 0) {
-            mbar_arrive_expect_tx(&q_land[1], QB);
+            if (!in_bounds(tile_row0(1) >= 0 && tile_row0(1) < p.N, kCheckQLoad)) {
+              ok = false;
+              *abort_flag = 1;
+              break;
+            }
+            q_issued[1] = true;
+            mbar_arrive_expect_tx(&q_full[1], QB);
             for (int c = 0; c < C::kChunks; ++c)
-              tma_load_3d(sQ + QB + c * kChunkBytes, &tmQ, &q_land[1], c * 64, tile_row0(1), bh);
+              tma_load_3d(sQ + QB + c * kChunkBytes, &tmQ, &q_full[1], c * 64, tile_row0(1), bh);
           }
         }
       }
@@ -350,35 +337,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // in shared memory after the CTA has ended.
         for (int s = 0; s < S && s < i; ++s) {
           const int last = s + ((i - 1 - s) / S) * S;
-          mbar_wait_drain<PAIR>(&kv_land[s], static_cast<uint32_t>(last / S) & 1u, tmo);
+          mbar_wait_drain(&kv_full[s], static_cast<uint32_t>(last / S) & 1u, tmo);
         }
-        if (tile_active[0]) mbar_wait_drain<PAIR>(&q_land[0], 0, tmo);
-        if (i > 0) mbar_wait_drain<PAIR>(&q_land[1], 0, tmo);
-      }
-    }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ forwarder (PAIR)
-    // Each copy of this CTA that lands is announced on the even CTA's
-    // barrier, in the producer's issue order: Q0, K0, Q1, V0, K1, V1, ...
-    if (PAIR && lane == 0) {
-      auto fwd = [&](uint64_t* land, uint64_t* full, uint32_t parity) {
-        if (!mbar_wait<PAIR>(land, parity, abort_flag, status, tmo, kSiteLand)) return false;
-        mbar_arrive_cluster(mapa_shared(smem_addr(full), 0));
-        return true;
-      };
-      bool ok = fwd(&q_land[0], &q_full[0], 0);
-      for (int i = 0; i < 2 * n_iter && ok; ++i) {
-        const int s = i % S;
-        ok = fwd(&kv_land[s], &kv_full[s], static_cast<uint32_t>(i / S) & 1u);
-        if (ok && i == 0) ok = fwd(&q_land[1], &q_full[1], 0);
+        for (int t = 0; t < 2; ++t)
+          if (q_issued[t]) mbar_wait_drain(&q_full[t], 0, tmo);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && rank == 0 && n_iter > 0) {
-      constexpr uint32_t kM = PAIR ? 2 * kBM : kBM;
-      constexpr uint32_t idS = idesc_bf16_f32(kM, BN, false);
-      constexpr uint32_t idO = idesc_bf16_f32(kM, D, true);
+    if (lane == 0 && n_iter > 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(kBM, BN, false);
+      constexpr uint32_t idO = idesc_bf16_f32(kBM, D, true);
       const uint32_t sq = smem_addr(sQ);
       const uint32_t skv = smem_addr(sKV);
       // The issuing thread is on the critical path between the softmax and
@@ -400,38 +369,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t boff = (kk >> 2) * C::kKChunkBytes + (kk & 3) * 32;
           const uint64_t ad = kAdvanceDesc ? a0 + (aoff >> 4) : sw128_desc(sq + t * QB + aoff, 16, 1024);
           const uint64_t bd = kAdvanceDesc ? b0 + (boff >> 4) : sw128_desc(skv + s * SB + boff, 16, 1024);
-          if (PAIR)
-            mma_ss_pair(tmem + t * BN, ad, bd, idS, kk > 0 ? 1u : 0u);
-          else
-            mma_ss(tmem + t * BN, ad, bd, idS, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + t * BN, ad, bd, idS, kk > 0 ? 1u : 0u);
         }
       };
       // O_t (+)= P_t V: A = P_t in TMEM (8 columns per 16 keys), B = V stage
       // stored d-contiguous (MN-major): 16 keys = 2 KB apart, d halves 16 KB apart.
-      auto issue_pv = [&](int t, int s, bool accumulate, int half) {
+      auto issue_pv = [&](int t, int s, bool accumulate) {
         const uint64_t v0 = sw128_desc(skv + s * SB, C::kVChunkBytes, 1024);
 #pragma unroll
-        for (int kk = half * (BN / 32); kk < (half + 1) * (BN / 32); ++kk) {
+        for (int kk = 0; kk < BN / 16; ++kk) {
           const uint64_t bd = kAdvanceDesc ? v0 + static_cast<uint32_t>(kk * (2048 >> 4))
                                            : sw128_desc(skv + s * SB + kk * 2048, C::kVChunkBytes, 1024);
           const uint32_t acc = (accumulate || kk > 0) ? 1u : 0u;
-          if (PAIR)
-            mma_ts_pair(tmem + C::kColO + t * D, tmem + t * BN + kk * 8, bd, idO, acc);
-          else
-            mma_ts(tmem + C::kColO + t * D, tmem + t * BN + kk * 8, bd, idO, acc);
+          mma_ts(tmem + C::kColO + t * D, tmem + t * BN + kk * 8, bd, idO, acc);
         }
       };
-      auto commit = [&](uint64_t* bar) {
-        if (PAIR)
-          mma_commit_pair_mc(bar, 0x3);
-        else
-          mma_commit(bar);
-      };
-      bool ok = mbar_wait<PAIR>(&kv_full[0], 0, abort_flag, status, tmo, kSiteKvFull);
+      auto commit = [&](uint64_t* bar) { mma_commit(bar); };
+      bool ok = mbar_wait(&kv_full[0], 0, abort_flag, status, tmo, kSiteKvFull);
       bool q_ready[2] = {false, false};
       for (int t = 0; t < 2 && ok; ++t) {
         if (first_it[t] != 0) continue;
-        ok = mbar_wait<PAIR>(&q_full[t], 0, abort_flag, status, tmo, kSiteQ);
+        ok = mbar_wait(&q_full[t], 0, abort_flag, status, tmo, kSiteQ);
         if (!ok) break;
         q_ready[t] = true;
         tc_fence_after();
@@ -443,34 +401,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int iv = 2 * it + 1, ik = 2 * it + 2;
         const int sv = iv % S, sk = ik % S;
         const bool last = it == n_iter - 1;
-        if (!(ok = mbar_wait<PAIR>(&kv_full[sv], static_cast<uint32_t>(iv / S) & 1u, abort_flag, status, tmo, kSiteKvFull))) break;
+        if (!(ok = mbar_wait(&kv_full[sv], static_cast<uint32_t>(iv / S) & 1u, abort_flag, status, tmo, kSiteKvFull))) break;
         bool k_ready = false;
         for (int t = 0; t < 2; ++t) {
           if (it >= first_it[t]) {
-            // P_t arrives whole on p_half[2t], or (kPH == 2) in two
-            // halves of 64 keys on p_half[2t] and p_half[2t+1], so that the
-            // first four K-steps of the PV product start while the softmax
-            // is still on the second half.
             const uint32_t ph = static_cast<uint32_t>(it - first_it[t]) & 1u;
             const bool acc = it > first_it[t];
-            if (!(ok = mbar_wait<PAIR>(&p_half[2 * t], ph, abort_flag, status, tmo, kSiteP + 2 * t))) break;
+            if (!(ok = mbar_wait(&p_full[t], ph, abort_flag, status, tmo, kSiteP + t))) break;
             FA_TRACE_MARK(0, it, 3 * t);
             tc_fence_after();
-            issue_pv(t, sv, acc, 0);
-            if (kPH == 2 &&
-                !(ok = mbar_wait<PAIR>(&p_half[2 * t + 1], ph, abort_flag, status, tmo, kSiteP + 2 * t + 1))) break;
-            tc_fence_after();
-            issue_pv(t, sv, true, 1);
+            issue_pv(t, sv, acc);
             FA_TRACE_MARK(0, it, 3 * t + 1);
             if (last) commit(&o_full[t]);
           }
           if (!last && it + 1 >= first_it[t]) {
             if (!k_ready) {
-              if (!(ok = mbar_wait<PAIR>(&kv_full[sk], static_cast<uint32_t>(ik / S) & 1u, abort_flag, status, tmo, kSiteKvFull))) break;
+              if (!(ok = mbar_wait(&kv_full[sk], static_cast<uint32_t>(ik / S) & 1u, abort_flag, status, tmo, kSiteKvFull))) break;
               k_ready = true;
             }
             if (!q_ready[t]) {
-              if (!(ok = mbar_wait<PAIR>(&q_full[t], 0, abort_flag, status, tmo, kSiteQ))) break;
+              if (!(ok = mbar_wait(&q_full[t], 0, abort_flag, status, tmo, kSiteQ))) break;
               q_ready[t] = true;
             }
             tc_fence_after();
@@ -484,11 +434,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!last) commit(&kv_empty[sk]);
       }
       // every MMA issued here has finished before TMEM is released
-      if (PAIR)
-        mma_commit_pair_mc(mma_done, 0x1);
-      else
-        mma_commit(mma_done);
-      mbar_wait_drain<PAIR>(mma_done, 0, tmo);
+      mma_commit(mma_done);
+      mbar_wait_drain(mma_done, 0, tmo);
     }
   } else if (warp >= kSoftmaxWarp0 && (QT == 2 || warp >= kSoftmaxWarp0 + 4)) {
     // ------------------------------------------------------------ softmax
@@ -522,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float l_sum = 0.f;        // running denominator relative to m_ref
     bool ok = true;
     if (p.debug & 1u) {
-      ok = __all_sync(0xffffffffu, mbar_wait<PAIR>(never, 0, abort_flag, status, tmo, kSiteDebug));
+      ok = __all_sync(0xffffffffu, mbar_wait(never, 0, abort_flag, status, tmo, kSiteDebug));
     }
     for (int it = first_it[t]; it < n_iter && ok; ++it) {
       const int li = it - first_it[t];
@@ -537,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       ok = __all_sync(0xffffffffu,
-                      mbar_wait<PAIR>(&s_full[t], static_cast<uint32_t>(li) & 1u, abort_flag, status, tmo, kSiteS));
+                      mbar_wait(&s_full[t], static_cast<uint32_t>(li) & 1u, abort_flag, status, tmo, kSiteS));
       if (!ok) break;
       const bool tr = lane == 0 && (warp & 3) == 0;
       if (tr) FA_TRACE_MARK(1 + t, it, 0);
@@ -588,57 +535,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_ref = m_tile;
       }
       const bool rescale_o = li > 0 && __any_sync(0xffffffffu, raise);
-      if (kPH == 2 && rescale_o) rescale_o_rows(tO, alpha);
       const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
       const float2 sl2v = make_float2(sl2, sl2);
       const float2 nm2 = make_float2(neg_m, neg_m);
       float2 ps2[kQ32];
-      // p = 2^(s * scale * log2 e - m) (the last kEmuPer32 columns of every
-      // 32 on the FMA pipe, the rest on MUFU), written as bf16 pairs over the
-      // first BN/2 columns of S_t in halves of 64 keys, published on
-      // p_half[2t] (whole tile) or, with kPH == 2, each half on its own
-      // barrier p_half[2t+h] as soon as it is in TMEM.
+      // p = 2^(s * scale * log2 e - m), written as bf16 pairs over the first
+      // BN/2 columns of S_t, 32 keys at a time, and published whole on
+      // p_full[t].
 #pragma unroll
-      for (int h = 0; h < BN / 64; ++h) {
-        constexpr int kLastH = BN / 64 - 1;
-        uint32_t pk[32];
+      for (int q = 0; q < kQ32; ++q) {
+        // keys [32q, 32q + 32) -> 16 columns of bf16 pairs at column 16q
+        uint32_t pk[16];
+        ps2[q] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int qq = 0; qq < 2; ++qq) {
-          const int q = 2 * h + qq;
-          ps2[q] = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const float2 x = ffma2(make_float2(__uint_as_float(sr[q][c]), __uint_as_float(sr[q][c + 1])),
-                                   sl2v, nm2);
-            float2 pv;
-            if (c >= 32 - kEmuPer32) {
-              pv = exp2_poly2(x);
-            } else {
-              pv.x = ex2_approx(x.x);
-              pv.y = ex2_approx(x.y);
-            }
-            ps2[q] = fadd2(ps2[q], pv);
-            pk[qq * 16 + (c >> 1)] = pack_bf16x2(pv.x, pv.y);
-          }
+        for (int c = 0; c < 32; c += 2) {
+          const float2 x = ffma2(make_float2(__uint_as_float(sr[q][c]), __uint_as_float(sr[q][c + 1])),
+                                 sl2v, nm2);
+          float2 pv;
+          pv.x = ex2_approx(x.x);
+          pv.y = ex2_approx(x.y);
+          ps2[q] = fadd2(ps2[q], pv);
+          pk[c >> 1] = round_pack_bf16x2(pv.x, pv.y);
         }
-        tmem_st32(tS + h * 32, pk);
-        // whole-P: the rescale waits until the scores have left the registers
-        if (kPH == 1 && h == kLastH && rescale_o) rescale_o_rows(tO, alpha);
-        if (kPH == 2 || h == kLastH) {
-          tmem_wait_st();
-          tc_fence_before();
-          uint64_t* pbar = &p_half[2 * t + ((kPH == 2 && h == 1) ? 1 : 0)];
-          if (PAIR) {
-            // one arrival per warp on the even CTA's barrier, after every
-            // lane's stores are complete and fenced
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster_relaxed(mapa_shared(smem_addr(pbar), 0));
-          } else {
-            mbar_arrive(pbar);
-          }
-        }
-        if (tr && h == 0) FA_TRACE_MARK(1 + t, it, 3);
+        tmem_st16(tS + q * 16, pk);
+        if (tr && q == kQ32 / 2 - 1) FA_TRACE_MARK(1 + t, it, 3);
       }
+      // the rescale waits until the scores have left the registers
+      if (rescale_o) rescale_o_rows(tO, alpha);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[t]);
       float2 psum;
       if constexpr (kQ32 == 4)
         psum = fadd2(fadd2(ps2[0], ps2[1]), fadd2(ps2[2], ps2[3]));
@@ -649,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ------------------------------------------------------------ epilogue
-    if (ok && tile_active[t]) ok = mbar_wait<PAIR>(&o_full[t], 0, abort_flag, status, tmo, kSiteO);
+    if (ok && tile_active[t]) ok = mbar_wait(&o_full[t], 0, abort_flag, status, tmo, kSiteO);
     const bool failed = named_bar_or(1 + t, kBM, !ok);
     if (!failed && SPLIT) {
       // partial state of this key range: u / l (fp32) and its LSE; a range
@@ -660,28 +586,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float lse_val = l_sum > 0.f ? (m_ref + log2f(l_sum)) * 0.69314718055994530942f : -INFINITY;
       const size_t prow = (static_cast<size_t>(split) * p.BH + bh) * p.N + row;
       float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D);
-      if (row < p.N) p.lse_part[prow] = lse_val;
+      const bool row_ok =
+          row < p.N &&
+          in_bounds(split < p.num_splits && bh < p.BH && prow < static_cast<size_t>(p.num_splits) * p.BH * p.N,
+                    kCheckPartial);
+      if (row_ok) p.lse_part[prow] = lse_val;
       if (tile_active[t]) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
           tmem_ld32(tO + c * 32, o);
           tmem_wait_ld();
-          if (row < p.N) {
+          if (row_ok) {
 #pragma unroll
             for (int g = 0; g < 8; ++g)
               dst[c * 8 + g] = make_float4(__uint_as_float(o[4 * g]) * inv_l, __uint_as_float(o[4 * g + 1]) * inv_l,
                                            __uint_as_float(o[4 * g + 2]) * inv_l, __uint_as_float(o[4 * g + 3]) * inv_l);
           }
         }
-      } else if (row < p.N) {
+      } else if (row_ok) {
 #pragma unroll
         for (int g = 0; g < D / 4; ++g) dst[g] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     } else if (!failed) {
       tc_fence_after();
       const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
-      if (p.lse != nullptr && row < p.N) {
+      if (p.lse != nullptr && row < p.N && in_bounds(bh < p.BH && row >= 0, kCheckLse)) {
         const float lse2 = l_sum > 0.f ? m_ref + log2f(l_sum) : -INFINITY;
         p.lse[static_cast<size_t>(bh) * p.N + row] = lse2 * 0.69314718055994530942f;
       }
@@ -707,14 +637,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           v.z = pack_bf16x2(__uint_as_float(o[8 * g + 4]) * inv_l, __uint_as_float(o[8 * g + 5]) * inv_l);
           v.w = pack_bf16x2(__uint_as_float(o[8 * g + 6]) * inv_l, __uint_as_float(o[8 * g + 7]) * inv_l);
           const int gran = ((c & 1) * 4 + g) ^ (r & 7);
-          *reinterpret_cast<uint4*>(rowp + gran * 16) = v;
+          if (in_bounds(rowp + gran * 16 >= stage && rowp + gran * 16 + 16 <= stage + QB, kCheckStage))
+            *reinterpret_cast<uint4*>(rowp + gran * 16) = v;
         }
       }
       fence_proxy_async_smem();
       named_bar_sync(1 + t, kBM);
       if (r == 0 && row0 < p.N) {
         for (int c = 0; c < C::kChunks; ++c)
-          tma_store_3d(&tmO, stage + c * kChunkBytes, c * 64, row0, bh);
+          if (in_bounds(row0 >= 0 && bh < p.BH, kCheckStore))
+            tma_store_3d(&tmO, stage + c * kChunkBytes, c * 64, row0, bh);
         bulk_commit_group();
         bulk_wait_group_read0();
       }
@@ -722,17 +654,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   tc_fence_before();
-  if (PAIR)
-    cluster_sync();
-  else
-    __syncthreads();
+  __syncthreads();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    if (PAIR)
-      tmem_dealloc_pair(tmem, kTmemCols);
-    else
-      tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -758,6 +684,7 @@ __global__ void __launch_bounds__(256)
   for (int i = 0; i < kPer; ++i) acc[i] = 0.f;
   float wsum = 0.f;
   for (int s = 0; s < num_splits; ++s) {
+    if (!in_bounds(s * rows + row < num_splits * rows, kCheckMerge)) break;
     const float l = lse_part[s * rows + row];
     const float w = (l == -INFINITY) ? 0.f : ex2_approx((l - m) * 1.4426950408889634f);
     wsum += w;
@@ -798,67 +725,49 @@ using host::g_debug_flags;
 using host::g_last_error;
 using host::g_timeout_ns;
 using host::kDefaultTimeoutNs;
-using host::make_map;
+using host::make_map_cached;
 using host::overlaps;
 
+// Per-device facts found on first use.  No lock is held while launching: the
+// attribute call is idempotent, so two threads that both find it unset both
+// make it, harmlessly.
 struct DeviceInfo {
-  bool checked = false;
-  bool sm100 = false;
-  bool attr_set[128] = {};
+  std::atomic<int> sm100{0};  // 0 unknown, 1 yes, -1 no
+  std::atomic<bool> attr_set[128] = {};
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_devices[kMaxDevices];
-std::mutex g_dev_mutex;
-
-// The pair kernel (clusters of two CTAs, M = 256 MMAs) is built for d = 128
-// only when FA_PAIR is defined: on B200 it measured slower than one CTA per
-// block (the two SMs' softmax steps gate every shared MMA).
-#ifdef FA_PAIR
-template <int D>
-constexpr bool kUsePair = (D == 128);
-#else
-template <int D>
-constexpr bool kUsePair = false;
-#endif
 
 template <int D, bool CAUSAL, bool SPLIT, bool SPARSE = false, int BN = kBN, int QT = kQTiles>
 fa_status launch(const void* Q, const void* K, const void* V, void* O, FwdParams prm, int N, int BH,
                  cudaStream_t stream, DeviceInfo& dev) {
-  constexpr bool PAIR = kUsePair<D> && !SPLIT && !SPARSE && BN == kBN;
-  using C = Cfg<D, PAIR, BN>;
+  using C = Cfg<D, BN>;
   prm.n_kv = (N + BN - 1) / BN;
   CUtensorMap mq, mk, mv, mo;
-  if (!make_map(&mq, Q, D, N, BH, kBM) || !make_map(&mk, K, D, N, BH, C::kKRows) ||
-      !make_map(&mv, V, D, N, BH, BN) || !make_map(&mo, O, D, N, BH, kBM)) {
+  if (!make_map_cached(&mq, Q, D, N, BH, kBM) || !make_map_cached(&mk, K, D, N, BH, BN) ||
+      !make_map_cached(&mv, V, D, N, BH, BN) || !make_map_cached(&mo, O, D, N, BH, kBM)) {
     snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed");
     return FA_ERR_CUDA;
   }
-  const long long rows_per_block = static_cast<long long>(QT) * C::kRowsPerTile;
+  const long long rows_per_block = static_cast<long long>(QT) * kBM;
   prm.n_qblk = static_cast<int>((N + rows_per_block - 1) / rows_per_block);
   const long long units = static_cast<long long>(BH) * prm.n_qblk;
-  const long long grid = units * (SPLIT ? prm.num_splits : (PAIR ? 2 : 1));
+  const long long grid = units * (SPLIT ? prm.num_splits : 1);
   if (grid > 0x7fffffffll) return FA_ERR_SHAPE;
   constexpr int slot = (QT == 1 ? 64 : 0) + (BN == 64 ? 32 : 0) + (SPARSE ? 16 : 0) + (D == 128 ? 8 : 0) +
-                       (CAUSAL ? 4 : 0) + (PAIR ? 2 : 0) + (SPLIT ? 1 : 0);
-  auto kern = fa_fwd_kernel<D, CAUSAL, PAIR, SPLIT, SPARSE, BN, QT>;
-  if (!dev.attr_set[slot]) {
+                       (CAUSAL ? 4 : 0) + (SPLIT ? 1 : 0);
+  auto kern = fa_fwd_kernel<D, CAUSAL, SPLIT, SPARSE, BN, QT>;
+  if (!dev.attr_set[slot].load(std::memory_order_acquire)) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-    dev.attr_set[slot] = true;
+    dev.attr_set[slot].store(true, std::memory_order_release);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = PAIR ? 2 : 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, prm);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
@@ -897,6 +806,7 @@ const char* fa_status_string(fa_status s) {
     case FA_ERR_ALIAS: return "FA_ERR_ALIAS: O, LSE or the workspace overlaps an input or each other";
     case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: the workspace is smaller than required";
     case FA_ERR_LAYOUT: return "FA_ERR_LAYOUT: a block-sparse list was out of range or out of order";
+    case FA_ERR_BOUNDS: return "FA_ERR_BOUNDS: an index check of the debug build failed";
   }
   return "unknown fa_status";
 }
@@ -954,18 +864,14 @@ fa_status prepare(const float* LSE, int B, int H, int N, int d, float scale, Fwd
   cudaError_t e = cudaGetDevice(&dev_id);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev_id < 0 || dev_id >= kMaxDevices) return FA_ERR_UNSUPPORTED;
-  {
-    std::lock_guard<std::mutex> lock(g_dev_mutex);
-    *dev = &g_devices[dev_id];
-    if (!(*dev)->checked) {
-      int major = 0;
-      e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev_id);
-      if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
-      (*dev)->sm100 = (major == 10);
-      (*dev)->checked = true;
-    }
+  *dev = &g_devices[dev_id];
+  if ((*dev)->sm100.load(std::memory_order_acquire) == 0) {
+    int major = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev_id);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    (*dev)->sm100.store(major == 10 ? 1 : -1, std::memory_order_release);
   }
-  if (!(*dev)->sm100) return FA_ERR_UNSUPPORTED;
+  if ((*dev)->sm100.load(std::memory_order_acquire) != 1) return FA_ERR_UNSUPPORTED;
 
   *prm = FwdParams{};
   prm->lse = const_cast<float*>(LSE);
@@ -1008,6 +914,23 @@ int default_splits(int B, int H, int N, bool causal) {
   return static_cast<int>(s < 1 ? 1 : s);
 }
 
+// The range count a split-KV call really runs: num_splits <= 0 picks the
+// default; ranges are ceil(n_kv / num_splits) key tiles each, and trailing
+// empty ranges are dropped.  0 when num_splits exceeds kMaxSplits.
+int effective_splits(int B, int H, int N, bool causal, int num_splits) {
+  if (num_splits <= 0) num_splits = default_splits(B, H, N, causal);
+  if (num_splits > kMaxSplits) return 0;
+  const int n_kv = (N + kBN - 1) / kBN;
+  const int kv_per_split = (n_kv + num_splits - 1) / num_splits;
+  return (n_kv + kv_per_split - 1) / kv_per_split;
+}
+
+// Workspace bytes of a split-KV call that runs `splits` ranges: none for a
+// single range (the fused kernel writes O and LSE directly).
+size_t splitkv_need(int B, int H, int N, int d, int splits) {
+  return splits > 1 ? splitkv_bytes(B, H, N, d, splits) : 0;
+}
+
 }  // namespace
 }  // namespace fa
 
@@ -1023,7 +946,6 @@ fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
   if (st0 != FA_OK) return st0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int bh = prm.BH;
-  std::lock_guard<std::mutex> lock(g_dev_mutex);
   if (d == 128)
     return causal ? launch<128, true, false>(Q, K, V, O, prm, N, bh, st, *dev)
                   : launch<128, false, false>(Q, K, V, O, prm, N, bh, st, *dev);
@@ -1048,7 +970,6 @@ fa_status fa_fwd_tile_config(const void* Q, const void* K, const void* V, void* 
   if (st0 != FA_OK) return st0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int bh = prm.BH;
-  std::lock_guard<std::mutex> lock(g_dev_mutex);
   // (query rows, key tile) in {(256, 64), (128, 128), (128, 64)}; (256, 128) is fa_fwd
   if (query_rows == 256) {
     if (d == 128)
@@ -1079,9 +1000,8 @@ int fa_fwd_splitkv_default_splits(int B, int H, int N, int d, int causal) {
 
 size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int N, int d, int causal, int num_splits) {
   if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
-  if (num_splits <= 0) num_splits = fa::default_splits(B, H, N, causal != 0);
-  if (num_splits > fa::kMaxSplits) return 0;
-  return fa::splitkv_bytes(B, H, N, d, num_splits);
+  const int splits = fa::effective_splits(B, H, N, causal != 0, num_splits);
+  return splits == 0 ? 0 : fa::splitkv_need(B, H, N, d, splits);
 }
 
 fa_status fa_fwd_splitkv(const void* Q, const void* K, const void* V, void* O, float* LSE,
@@ -1092,28 +1012,28 @@ fa_status fa_fwd_splitkv(const void* Q, const void* K, const void* V, void* O, f
   DeviceInfo* dev = nullptr;
   fa_status st0 = check_args(Q, K, V, O, LSE, B, H, N, d, scale);
   if (st0 != FA_OK) return st0;
-  if (workspace == nullptr) return FA_ERR_NULL;
-  if ((reinterpret_cast<uintptr_t>(workspace) & 15u) != 0) return FA_ERR_ALIGN;
-  if (num_splits <= 0) num_splits = default_splits(B, H, N, causal != 0);
-  if (num_splits > kMaxSplits) return FA_ERR_UNSUPPORTED;
   // equal ranges of key tiles; trailing empty ranges are dropped
+  num_splits = effective_splits(B, H, N, causal != 0, num_splits);
+  if (num_splits == 0) return FA_ERR_UNSUPPORTED;
   const int n_kv = (N + kBN - 1) / kBN;
   const int kv_per_split = (n_kv + num_splits - 1) / num_splits;
-  num_splits = (n_kv + kv_per_split - 1) / kv_per_split;
-  const size_t need = splitkv_bytes(B, H, N, d, num_splits);
-  if (workspace_bytes < need) return FA_ERR_WORKSPACE;
-  const size_t nbytes = static_cast<size_t>(B) * H * N * d * 2;
-  if (overlaps(workspace, need, Q, nbytes) || overlaps(workspace, need, K, nbytes) ||
-      overlaps(workspace, need, V, nbytes) || overlaps(workspace, need, O, nbytes) ||
-      (LSE && overlaps(workspace, need, LSE, static_cast<size_t>(B) * H * N * 4)))
-    return FA_ERR_ALIAS;
+  const size_t need = splitkv_need(B, H, N, d, num_splits);
+  if (need > 0) {
+    if (workspace == nullptr) return FA_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 15u) != 0) return FA_ERR_ALIGN;
+    if (workspace_bytes < need) return FA_ERR_WORKSPACE;
+    const size_t nbytes = static_cast<size_t>(B) * H * N * d * 2;
+    if (overlaps(workspace, need, Q, nbytes) || overlaps(workspace, need, K, nbytes) ||
+        overlaps(workspace, need, V, nbytes) || overlaps(workspace, need, O, nbytes) ||
+        (LSE && overlaps(workspace, need, LSE, static_cast<size_t>(B) * H * N * 4)))
+      return FA_ERR_ALIAS;
+  }
   st0 = prepare(LSE, B, H, N, d, scale, &prm, &dev);
   if (st0 != FA_OK) return st0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int bh = prm.BH;
   if (num_splits == 1) {
     // one range: the fused kernel writes O and LSE directly
-    std::lock_guard<std::mutex> lock(g_dev_mutex);
     if (d == 128)
       return causal ? launch<128, true, false>(Q, K, V, O, prm, N, bh, st, *dev)
                     : launch<128, false, false>(Q, K, V, O, prm, N, bh, st, *dev);
@@ -1125,7 +1045,6 @@ fa_status fa_fwd_splitkv(const void* Q, const void* K, const void* V, void* O, f
   prm.kv_per_split = kv_per_split;
   prm.o_part = static_cast<float*>(workspace);
   prm.lse_part = prm.o_part + static_cast<size_t>(num_splits) * rows * d;
-  std::lock_guard<std::mutex> lock(g_dev_mutex);
   fa_status r;
   if (d == 128)
     r = causal ? launch<128, true, true>(Q, K, V, O, prm, N, bh, st, *dev)
@@ -1165,7 +1084,6 @@ fa_status fa_fwd_block_sparse(const void* Q, const void* K, const void* V, void*
   prm.blk_nnz = nnz;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int bh = prm.BH;
-  std::lock_guard<std::mutex> lock(g_dev_mutex);
   if (d == 128)
     return causal ? launch<128, true, false, true>(Q, K, V, O, prm, N, bh, st, *dev)
                   : launch<128, false, false, true>(Q, K, V, O, prm, N, bh, st, *dev);
@@ -1210,8 +1128,10 @@ fa_status fa_fwd_splitkv_noalloc(const void* Q, const void* K, const void* V, vo
   // argument errors are reported exactly as fa_fwd_splitkv reports them
   fa_status st0 = check_args(Q, K, V, O, LSE, B, H, N, d, scale);
   if (st0 != FA_OK) return st0;
-  if (num_splits > kMaxSplits) return FA_ERR_UNSUPPORTED;
-  const size_t need = fa_fwd_splitkv_workspace_bytes(B, H, N, d, causal, num_splits);
+  // the ranges this call really runs: a single range needs no scratch at all
+  const int splits = effective_splits(B, H, N, causal != 0, num_splits);
+  if (splits == 0) return FA_ERR_UNSUPPORTED;
+  const size_t need = splitkv_need(B, H, N, d, splits);
   if (need > static_cast<size_t>(FA_NOALLOC_SCRATCH_BYTES)) return FA_ERR_WORKSPACE;
   int dev_id = 0;
   cudaError_t e = cudaGetDevice(&dev_id);
@@ -1233,7 +1153,7 @@ fa_status fa_fwd_splitkv_noalloc(const void* Q, const void* K, const void* V, vo
   // Every partial state the merge reads is written first by the same call,
   // so nothing in the scratch has to start at zero.
   return fa_fwd_splitkv(Q, K, V, O, LSE, scratch, static_cast<size_t>(FA_NOALLOC_SCRATCH_BYTES), B,
-                        H, N, d, scale, causal, num_splits, stream);
+                        H, N, d, scale, causal, splits, stream);
 }
 
 fa_status fa_get_device_status_word(void* stream, unsigned int* word) {
@@ -1253,7 +1173,8 @@ fa_status fa_get_device_status_word(void* stream, unsigned int* word) {
     const uint32_t zero = 0;
     e = cudaMemcpyToSymbol(fa::g_device_status, &zero, sizeof(zero));  // backward's already cleared
     if (e != cudaSuccess) return fa::cuda_fail(e, "cudaMemcpyToSymbol");
-    return (v & fa::kStatusTimeout) ? FA_ERR_DEVICE_TIMEOUT : FA_ERR_LAYOUT;
+    if (v & fa::kStatusTimeout) return FA_ERR_DEVICE_TIMEOUT;
+    return (v & fa::kStatusBounds) ? FA_ERR_BOUNDS : FA_ERR_LAYOUT;
   }
   return FA_OK;
 }

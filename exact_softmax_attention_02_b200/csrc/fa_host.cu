@@ -144,6 +144,20 @@ fa_status fa_fwd_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, 
   ck(cudaStreamWaitEvent(p.comp, p.start, 0), "cudaStreamWaitEvent");
   ck(cudaStreamWaitEvent(p.d2h, p.start, 0), "cudaStreamWaitEvent");
   if (e != cudaSuccess) return FA_ERR_CUDA;
+  // On an error after work was enqueued: join all three streams back into the
+  // caller's stream before returning, so that no copy into the caller's host
+  // buffers and no read of the workspace outlives what the caller's stream
+  // orders after this call.  Errors of these joining calls are not reported
+  // over the first one.
+  auto fail = [&](fa_status result) {
+    cudaEventRecord(p.start, p.h2d);
+    cudaStreamWaitEvent(p.d2h, p.start, 0);
+    cudaEventRecord(p.start, p.comp);
+    cudaStreamWaitEvent(p.d2h, p.start, 0);
+    cudaEventRecord(p.done, p.d2h);
+    cudaStreamWaitEvent(caller, p.done, 0);
+    return result;
+  };
   for (int c = 0; c < chunks; ++c) {
     const long long h0 = c * per, h1 = (h0 + per < BH) ? h0 + per : BH;
     const size_t off = static_cast<size_t>(h0) * head_bytes;
@@ -153,11 +167,11 @@ fa_status fa_fwd_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, 
     ck(cudaMemcpyAsync(Vd + off, vh + off, len, cudaMemcpyHostToDevice, p.h2d), "cudaMemcpyAsync V");
     ck(cudaEventRecord(p.in[c], p.h2d), "cudaEventRecord");
     ck(cudaStreamWaitEvent(p.comp, p.in[c], 0), "cudaStreamWaitEvent");
-    if (e != cudaSuccess) return FA_ERR_CUDA;
+    if (e != cudaSuccess) return fail(FA_ERR_CUDA);
     // the heads of this chunk are one [1][h1-h0][N][d] problem
     st = fa_fwd(Qd + off, Kd + off, Vd + off, Od + off, LSEh ? Ld + h0 * N : nullptr, 1,
                 static_cast<int>(h1 - h0), N, d, scale, causal, p.comp);
-    if (st != FA_OK) return st;
+    if (st != FA_OK) return fail(st);
     ck(cudaEventRecord(p.kern[c], p.comp), "cudaEventRecord");
     ck(cudaStreamWaitEvent(p.d2h, p.kern[c], 0), "cudaStreamWaitEvent");
     ck(cudaMemcpyAsync(oh + off, Od + off, len, cudaMemcpyDeviceToHost, p.d2h), "cudaMemcpyAsync O");
@@ -165,7 +179,7 @@ fa_status fa_fwd_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, 
       ck(cudaMemcpyAsync(LSEh + h0 * N, Ld + h0 * N, static_cast<size_t>(h1 - h0) * N * 4,
                          cudaMemcpyDeviceToHost, p.d2h),
          "cudaMemcpyAsync LSE");
-    if (e != cudaSuccess) return FA_ERR_CUDA;
+    if (e != cudaSuccess) return fail(FA_ERR_CUDA);
   }
   // the caller's stream resumes once every copy out has landed
   ck(cudaEventRecord(p.done, p.d2h), "cudaEventRecord");

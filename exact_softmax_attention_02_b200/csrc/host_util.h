@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstdio>
 #include <mutex>
@@ -57,6 +58,44 @@ inline bool make_map(CUtensorMap* map, const void* base, int d, int N, int BH, i
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// make_map through a small per-thread cache.  A tensor map holds only the
+// base address, the extents, the strides and the box, so an entry keyed by
+// exactly those stays valid for as long as the process runs, whatever happens
+// to the memory in between (a buffer freed and reallocated at the same address
+// with the same shape gets the same map).  Per thread, so no lock is taken.
+inline bool make_map_cached(CUtensorMap* map, const void* base, int d, int N, int BH, int box_rows) {
+  struct Entry {
+    const void* base;
+    int d, N, BH, box_rows;
+    unsigned stamp;
+    CUtensorMap map;
+  };
+  constexpr int kEntries = 16;
+  thread_local Entry cache[kEntries] = {};
+  thread_local unsigned clock = 0;
+  if (++clock == 0) ++clock;  // 0 marks an empty entry
+  int victim = 0;
+  for (int i = 0; i < kEntries; ++i) {
+    Entry& e = cache[i];
+    if (e.stamp != 0 && e.base == base && e.d == d && e.N == N && e.BH == BH && e.box_rows == box_rows) {
+      e.stamp = clock;
+      *map = e.map;
+      return true;
+    }
+    if (e.stamp < cache[victim].stamp) victim = i;
+  }
+  if (!make_map(map, base, d, N, BH, box_rows)) return false;
+  Entry& e = cache[victim];
+  e.base = base;
+  e.d = d;
+  e.N = N;
+  e.BH = BH;
+  e.box_rows = box_rows;
+  e.stamp = clock;
+  e.map = *map;
+  return true;
 }
 
 inline bool overlaps(const void* a, size_t na, const void* b, size_t nb) {

@@ -44,28 +44,15 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
-// kCluster: acquire at cluster scope, for barriers that other CTAs of the
-// cluster arrive on (remote arrivals, multicast commits).
-template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t done;
-  if (kCluster) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(bar), "r"(parity)
-        : "memory");
-  } else {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(bar), "r"(parity)
-        : "memory");
-  }
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
   return done != 0;
 }
 
@@ -73,6 +60,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 enum : uint32_t {
   kStatusTimeout = 1u,  // a bounded wait gave up
   kStatusLayout = 2u,   // a block-sparse list was malformed
+  kStatusBounds = 4u,   // an index check of a FA_DEBUG build failed
 };
 
 // Wait until the phase with the given parity has completed.  Gives up (and
@@ -80,14 +68,13 @@ enum : uint32_t {
 // global time, in which case it sets *abort itself and raises, in *status,
 // the timeout bit and bit 8 + site (site < 24 names the wait that gave up).
 // Never traps.
-template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint32_t* status, uint64_t timeout_ns, uint32_t site) {
   const uint32_t a = smem_addr(bar);
-  if (mbar_try_wait<kCluster>(a, parity)) return true;
+  if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait<kCluster>(a, parity)) return true;
+    if (mbar_try_wait(a, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
       if (global_timer_ns() - t0 > timeout_ns) {
@@ -100,12 +87,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // Same wait, ignoring the abort flag: used only while draining copies in flight.
-template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
   const uint32_t a = smem_addr(bar);
   const uint64_t t0 = global_timer_ns();
   for (;;) {
-    if (mbar_try_wait<kCluster>(a, parity)) return true;
+    if (mbar_try_wait(a, parity)) return true;
     if (global_timer_ns() - t0 > timeout_ns) return false;
   }
 }
@@ -353,92 +339,6 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 }
 
 // ---------------------------------------------------------------------------
-// clusters of two CTAs sharing one MMA (cta_group::2)
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-// All threads of every CTA of the cluster: release prior writes, wait for all.
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
-}
-
-// shared::cluster address of the same shared variable in CTA `rank`.
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
-
-// Arrive on an mbarrier that may live in another CTA of the cluster.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-
-// Same, without release semantics: for signals whose data is ordered by other
-// means (tensor-memory stores ordered by tcgen05.wait::st and
-// tcgen05.fence::before_thread_sync), so no generic-memory fence is paid.
-__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-
-// Both CTAs of the pair (same warp in each): allocate the same TMEM columns.
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t* slot, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                   smem_addr(slot)),
-               "r"(ncols)
-               : "memory");
-}
-
-__device__ __forceinline__ void tmem_relinquish_pair() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-
-// M = 256 MMA over the pair, issued by the even CTA: A rows 0-127 and the
-// first half of B's N come from the even CTA, the rest from the odd one; D
-// rows land in each CTA's own TMEM.
-__device__ __forceinline__ void mma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void mma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Arrive once, on the mbarrier at the same shared offset in every CTA of
-// `cta_mask`, when all pair MMAs issued so far by this thread have completed.
-__device__ __forceinline__ void mma_commit_pair_mc(uint64_t* bar, uint16_t cta_mask) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
-      "[%0], %1;" ::"r"(smem_addr(bar)),
-      "h"(cta_mask)
-      : "memory");
-}
-
-// ---------------------------------------------------------------------------
 // math
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -481,30 +381,19 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   return bits_f2(d);
 }
 
-// 2^x on the FMA pipe, for x <= 64: 2^x = 2^j 2^f with j = round(x),
-// f = x - j in [-1/2, 1/2], 2^f from a degree-3 polynomial of minimax
-// relative error 7.5e-5 (coefficients from csrc/fit_exp2.py), and 2^j added
-// into the exponent field.  Inputs below -126 (including -inf) are clamped,
-// giving a value below 2^-126 instead of 0.
-constexpr float kExp2C0 = 0.999928057f;
-constexpr float kExp2C1 = 0.693260968f;
-constexpr float kExp2C2 = 0.242610931f;
-constexpr float kExp2C3 = 0.0551714934f;
-constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
-
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -126.0f);
-  x.y = fmaxf(x.y, -126.0f);
-  const float2 t = fadd2(x, make_float2(kRoundMagic, kRoundMagic));  // j in the low mantissa bits
-  const float2 j = fadd2(t, make_float2(-kRoundMagic, -kRoundMagic));
-  const float2 f = fadd2(x, make_float2(-j.x, -j.y));
-  float2 p = ffma2(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
-  p = ffma2(p, f, make_float2(kExp2C1, kExp2C1));
-  p = ffma2(p, f, make_float2(kExp2C0, kExp2C0));
-  // (bits(t) << 23) == j << 23 modulo 2^32: the exponent increment
-  const uint32_t ex = __float_as_uint(p.x) + (__float_as_uint(t.x) << 23);
-  const uint32_t ey = __float_as_uint(p.y) + (__float_as_uint(t.y) << 23);
-  return make_float2(__uint_as_float(ex), __uint_as_float(ey));
+// Two floats to a bf16 pair (lo in bits 0-15) rounded to nearest, ties away
+// from zero, in integer arithmetic: adding half a unit of the last kept place
+// (0x8000) to each bit pattern carries into the kept 16 bits exactly when the
+// dropped 16 bits are at least half a unit, and one byte permute keeps the two
+// high halves.  It differs from round-to-nearest-even only on exact ties.
+// Infinities stay infinite and finite values past the largest bf16 become
+// infinite, as with round-to-nearest; NaN inputs give an undefined result.
+// On B200 this runs on the integer pipe.  The converting instruction
+// (cvt.rn.bf16x2.f32) applied to results of ex2.approx measured about 16
+// cycles per warp instruction in the softmax loop instead of 2, doubling the
+// loop's time, so the hot loops pack with this form.
+__device__ __forceinline__ uint32_t round_pack_bf16x2(float lo, float hi) {
+  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -45,7 +45,15 @@ def _load():
     global _lib
     if _lib is not None:
         return _lib
-    path = library_path()
+    _lib = load_library(library_path())
+    return _lib
+
+
+def load_library(path: str):
+    """Open a build of libfa.so at ``path`` and declare its signatures.
+
+    ``_load`` uses this for the library the module calls; the debug-build tests
+    use it to open ``libfa_debug.so`` beside it."""
     if not os.path.exists(path):
         raise RuntimeError(
             f"{path} not found: build the CUDA library first "
@@ -88,7 +96,6 @@ def _load():
     lib.fa_fwd_host_workspace_bytes.restype = ctypes.c_size_t
     lib.fa_version.argtypes = []
     lib.fa_version.restype = ctypes.c_char_p
-    _lib = lib
     return lib
 
 

@@ -43,7 +43,8 @@ typedef enum fa_status {
   FA_ERR_DEVICE_TIMEOUT = 6,  /* a kernel gave up on a bounded wait               */
   FA_ERR_ALIAS = 7,           /* O, LSE or a workspace overlaps another argument  */
   FA_ERR_WORKSPACE = 8,       /* the workspace is smaller than required           */
-  FA_ERR_LAYOUT = 9           /* a block-sparse list was out of range or order    */
+  FA_ERR_LAYOUT = 9,          /* a block-sparse list was out of range or order    */
+  FA_ERR_BOUNDS = 10          /* an index check of the debug build failed          */
 } fa_status;
 
 /*
@@ -90,23 +91,27 @@ fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
  *                    least fa_fwd_splitkv_workspace_bytes(B, H, N, d,
  *                    causal, num_splits) bytes; overwritten (fp32 partial outputs
  *                    [splits][B*H*N][d] followed by partial LSE
- *                    [splits][B*H*N]); must not overlap any other argument.
+ *                    [splits][B*H*N], splits = the ranges that remain, below);
+ *                    must not overlap any other argument.  When one range
+ *                    remains it is not used at all and may be NULL.
  *   workspace_bytes  its size.
  *   num_splits       1..256; <= 0 picks fa_fwd_splitkv_default_splits().
  *                    Ranges are ceil(ceil(N/128) / num_splits) key tiles;
  *                    trailing empty ranges are dropped.  When one range
- *                    remains, the fused kernel of fa_fwd runs and the
- *                    workspace is not touched.
- * Errors as fa_fwd, plus FA_ERR_NULL for a NULL workspace, FA_ERR_ALIGN for a
- * misaligned one, FA_ERR_WORKSPACE when it is too small, FA_ERR_UNSUPPORTED
- * for num_splits > 256.  Two kernels are enqueued on `stream`.
+ *                    remains, the fused kernel of fa_fwd runs alone.
+ * Errors as fa_fwd, plus (only when more than one range remains) FA_ERR_NULL
+ * for a NULL workspace, FA_ERR_ALIGN for a misaligned one, FA_ERR_WORKSPACE
+ * when it is too small; FA_ERR_UNSUPPORTED for num_splits > 256.  Two kernels
+ * are enqueued on `stream` (one when a single range remains).
  */
 fa_status fa_fwd_splitkv(const void* Q, const void* K, const void* V, void* O, float* LSE,
                          void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
                          float scale, int causal, int num_splits, void* stream);
 
-/* Bytes of workspace fa_fwd_splitkv needs (0 for invalid arguments).
- * num_splits <= 0 means the default for this shape and mask. */
+/* Bytes of workspace fa_fwd_splitkv needs for the ranges that remain after
+ * empty ones are dropped: 0 when a single range remains (no workspace is
+ * used) and 0 for invalid arguments.  num_splits <= 0 means the default for
+ * this shape and mask. */
 size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int N, int d, int causal, int num_splits);
 
 /* Default split count: non-causal, the most ranges that fit in one wave of
@@ -160,9 +165,10 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N);
  * exits.  The caller still passes Q, K, V, O and LSE, with the meaning,
  * layout and errors of fa_fwd_splitkv (num_splits <= 0 picks the default).
  *
- *   - A problem whose workspace (fa_fwd_splitkv_workspace_bytes) exceeds
- *     FA_NOALLOC_SCRATCH_BYTES is rejected with FA_ERR_WORKSPACE before
- *     anything is enqueued.
+ *   - A problem whose workspace (fa_fwd_splitkv_workspace_bytes, counted
+ *     for the ranges that remain) exceeds FA_NOALLOC_SCRATCH_BYTES is
+ *     rejected with FA_ERR_WORKSPACE before anything is enqueued.  A problem
+ *     that runs as a single range needs none and is never rejected for size.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current) and keeps it; make
  *     that first call before any stream capture.  The library allocates
@@ -172,6 +178,9 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N);
  *     that may overlap on the GPU -- on different streams without ordering,
  *     or from several host threads -- race on it and must be serialised by
  *     the caller.
+ *   - After fa_get_device_status() reports FA_ERR_DEVICE_TIMEOUT for such a
+ *     call, O and LSE are undefined and may hold values merged from partial
+ *     states an earlier call left in the array.
  */
 fa_status fa_fwd_splitkv_noalloc(const void* Q, const void* K, const void* V, void* O, float* LSE,
                                  int B, int H, int N, int d, float scale, int causal, int num_splits,
@@ -296,17 +305,20 @@ const char* fa_status_string(fa_status status);
  * device status words (forward and backward kernels) of the current device.
  * Returns FA_ERR_DEVICE_TIMEOUT
  * if any kernel launched by this library gave up on a bounded wait since the
- * last call (its outputs are then undefined), FA_ERR_LAYOUT if a
- * block-sparse call met a malformed list (and no wait gave up), FA_ERR_CUDA
- * if the synchronisation failed, FA_OK otherwise.
+ * last call (its outputs are then undefined), FA_ERR_BOUNDS if, in a library
+ * built with -DFA_DEBUG, an index check failed (the access was skipped and
+ * the outputs are undefined), FA_ERR_LAYOUT if a block-sparse call met a
+ * malformed list (and nothing else failed), FA_ERR_CUDA if the
+ * synchronisation failed, FA_OK otherwise.
  */
 fa_status fa_get_device_status(void* stream);
 
 /*
  * fa_get_device_status_word -- as fa_get_device_status, and also stores the
  * raw status word in *word (0 = no failure; bit 0 = a wait gave up; bit 1 = a
- * malformed block-sparse list; bit 8+k = the wait at site k gave up, for
- * diagnosis).  word may be NULL.
+ * malformed block-sparse list; bit 2 = an index check of a debug build
+ * failed; bit 8+k = the wait at site k gave up; bit 16+k = the index check
+ * at site k failed, for diagnosis).  word may be NULL.
  */
 fa_status fa_get_device_status_word(void* stream, unsigned int* word);
 

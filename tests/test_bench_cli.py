@@ -36,7 +36,7 @@ def test_unknown_experiment_is_rejected():
     assert "invalid choice" in r.stderr
 
 
-@pytest.mark.parametrize("experiment", ["sparse", "tiles", "library"])
+@pytest.mark.parametrize("experiment", ["sparse", "tiles"])
 def test_experiments_need_a_cuda_device(no_cuda, experiment):
     r = _bench("--experiment", experiment, "--steps", "3")
     assert r.returncode != 0

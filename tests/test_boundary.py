@@ -54,7 +54,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(10):
+    for code in range(11):
         s = lib.fa_status_string(code).decode()
         assert s.startswith("FA_")
     assert lib.fa_status_string(99).decode() == "unknown fa_status"
@@ -132,6 +132,11 @@ def test_splitkv_workspace_checks(lib):
     assert lib.fa_fwd_splitkv_workspace_bytes(1, 1, 1024, 96, 0, 2) == 0
     # the default split count depends on the mask
     assert lib.fa_fwd_splitkv_workspace_bytes(1, 2, 8192, 128, 1, 0) == 4 * 2 * 8192 * 129 * 4
+    # sized for the ranges that remain: 100 requested over 8 key tiles runs 8
+    assert lib.fa_fwd_splitkv_workspace_bytes(1, 1, 1024, 64, 0, 100) == 8 * 1024 * 65 * 4
+    # a single range runs the fused kernel alone and needs no workspace
+    assert lib.fa_fwd_splitkv_workspace_bytes(2, 16, 8192, 128, 1, 1) == 0
+    assert lib.fa_fwd_splitkv_workspace_bytes(1, 1, 100, 64, 0, 4) == 0
     assert _splitkv(lib, ws=None) == FA_ERR_NULL
     assert _splitkv(lib, ws=A + 512 * MB + 4) == FA_ERR_ALIGN
     assert _splitkv(lib, ws_bytes=need - 4) == FA_ERR_WORKSPACE

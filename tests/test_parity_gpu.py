@@ -93,10 +93,38 @@ def test_peaked_rows_stress_rescaling(d):
     compare(q, k, v, False, every_row(1, 4, 1024))
 
 
+def lse_accumulation_bound(q, k, scale, causal, rows):
+    """Per-row bound on |LSE_gpu - LSE_exact| for scores far outside N(0,1) scale.
+
+    LSE is 1-Lipschitz in the largest change of any one score, so its error is
+    at most max_j |ds_j| plus the error of the softmax steps.  The tensor core
+    sums the d exact bf16 products of a score in fp32; summing d terms in
+    fp32 errs by at most d * 2^-23 * sum_i |q_i k_ji| (the standard bound for
+    recursive summation, with one ulp per addition to allow truncating
+    rather than rounding adders).  Scaled, that is the second term; the first
+    is the tolerance of the N(0,1) regime, which covers the softmax steps.
+    For N(0,1) inputs at d = 128 the second term is about 1e-4."""
+    qa, ka = q.float().numpy().astype(np.float64), k.float().numpy().astype(np.float64)
+    d = q.shape[-1]
+    out = []
+    for b, h, i in rows:
+        n = i + 1 if causal else ka.shape[2]
+        mags = np.abs(ka[b, h, :n]) @ np.abs(qa[b, h, i])
+        out.append(1e-3 + d * 2.0 ** -23 * scale * mags.max())
+    return np.array(out)
+
+
 def test_large_score_magnitudes():
-    """Scores of several hundred: exponents must stay bounded (max subtraction)."""
+    """Scores of several hundred: exponents must stay bounded (max subtraction).
+
+    Q ~ N(0, 20^2) and K ~ N(0, 3^2) give scaled scores of standard deviation
+    60, so the fp32 accumulation of each score, not the softmax, limits the
+    LSE: the bound is derived per row (lse_accumulation_bound)."""
     q, k, v = make_qkv(1, 2, 512, 128, seed=5, q_std=20.0, k_std=3.0)
-    compare(q, k, v, True, every_row(1, 2, 512), lse_max=5e-3)
+    rows = every_row(1, 2, 512).numpy()
+    bound = lse_accumulation_bound(q, k, 1 / math.sqrt(128), True, rows)
+    _, _, _, lerr = compare(q, k, v, True, rows, lse_max=float("inf"))
+    assert np.all(lerr <= bound), f"max |dLSE| - bound = {(lerr - bound).max():.3e}"
 
 
 def test_custom_scale_and_no_lse():
