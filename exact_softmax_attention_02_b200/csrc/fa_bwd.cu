@@ -163,8 +163,8 @@ __device__ __forceinline__ void ds_16(const float (&p)[16], const uint32_t (&dp)
       const float2 pv = make_float2(p[e + u], p[e + u + 1]);
       const float2 g = fadd2(make_float2(__uint_as_float(dp[e + u]), __uint_as_float(dp[e + u + 1])), dv);
       const float2 dsv = fmul2(pv, g);
-      pk[(e + u) >> 1] = round_pack_bf16x2(pv.x, pv.y);
-      dk[(e + u) >> 1] = round_pack_bf16x2(dsv.x, dsv.y);
+      pk[(e + u) >> 1] = pack_bf16x2(pv.x, pv.y);
+      dk[(e + u) >> 1] = pack_bf16x2(dsv.x, dsv.y);
     }
   }
 }

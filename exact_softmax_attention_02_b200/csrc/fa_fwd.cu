@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       bool q_issued[2] = {false, false};
       if (tile_active[0]) {
-        if (in_bounds(tile_row0(0) >= 0 && tile_row0(0) < p.N && bh < p.BH, kCheckQLoad)) {
+        if (in_bounds(tile_row0(0) >= 0 && tile_row0(0) < p.n_qblk * QT * kBM && bh < p.BH, kCheckQLoad)) {
           q_issued[0] = true;
           mbar_arrive_expect_tx(&q_full[0], QB);
           for (int c = 0; c < C::kChunks; ++c)
@@ -320,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(st + c * C::kKChunkBytes, map, &kv_full[s], c * 64, j * BN, bh);
           ++i;
           if (it == 0 && kv == 0) {
-            if (!in_bounds(tile_row0(1) >= 0 && tile_row0(1) < p.N, kCheckQLoad)) {
+            if (!in_bounds(tile_row0(1) >= 0 && tile_row0(1) < p.n_qblk * QT * kBM, kCheckQLoad)) {
               ok = false;
               *abort_flag = 1;
               break;
@@ -540,25 +540,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float2 nm2 = make_float2(neg_m, neg_m);
       float2 ps2[kQ32];
       // p = 2^(s * scale * log2 e - m), written as bf16 pairs over the first
-      // BN/2 columns of S_t, 32 keys at a time, and published whole on
+      // BN/2 columns of S_t, 64 keys at a time, and published whole on
       // p_full[t].
 #pragma unroll
-      for (int q = 0; q < kQ32; ++q) {
-        // keys [32q, 32q + 32) -> 16 columns of bf16 pairs at column 16q
-        uint32_t pk[16];
-        ps2[q] = make_float2(0.f, 0.f);
+      for (int h = 0; h < BN / 64; ++h) {
+        // keys [64h, 64h + 64) -> 32 columns of bf16 pairs at column 32h
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const float2 x = ffma2(make_float2(__uint_as_float(sr[q][c]), __uint_as_float(sr[q][c + 1])),
-                                 sl2v, nm2);
-          float2 pv;
-          pv.x = ex2_approx(x.x);
-          pv.y = ex2_approx(x.y);
-          ps2[q] = fadd2(ps2[q], pv);
-          pk[c >> 1] = round_pack_bf16x2(pv.x, pv.y);
+        for (int qq = 0; qq < 2; ++qq) {
+          const int q = 2 * h + qq;
+          ps2[q] = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float2 x = ffma2(make_float2(__uint_as_float(sr[q][c]), __uint_as_float(sr[q][c + 1])),
+                                   sl2v, nm2);
+            float2 pv;
+            pv.x = ex2_approx(x.x);
+            pv.y = ex2_approx(x.y);
+            ps2[q] = fadd2(ps2[q], pv);
+            pk[qq * 16 + (c >> 1)] = pack_bf16x2(pv.x, pv.y);
+          }
         }
-        tmem_st16(tS + q * 16, pk);
-        if (tr && q == kQ32 / 2 - 1) FA_TRACE_MARK(1 + t, it, 3);
+        tmem_st32(tS + h * 32, pk);
+        if (tr && h == 0) FA_TRACE_MARK(1 + t, it, 3);
       }
       // the rescale waits until the scores have left the registers
       if (rescale_o) rescale_o_rows(tO, alpha);
@@ -839,7 +843,7 @@ fa_status check_args(const void* Q, const void* K, const void* V, const void* O,
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (!(scale > 0.f)) return FA_ERR_UNSUPPORTED;
   const long long BH = static_cast<long long>(B) * H;
-  const long long n_qblk = (static_cast<long long>(N) + kQTiles * kBM - 1) / (kQTiles * kBM);
+  const long long n_qblk = (static_cast<long long>(N) + kBM - 1) / kBM;  // 128-row query tiles (any kernel shape)
   if (BH > (1ll << 30) || BH * n_qblk > 0x7fffffffll) return FA_ERR_SHAPE;
   auto mis16 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) != 0; };
   if (mis16(Q) || mis16(K) || mis16(V) || mis16(O)) return FA_ERR_ALIGN;

@@ -56,6 +56,39 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 
+// As mbar_try_wait, but a thread whose phase is not complete is suspended
+// until it completes or about `hint_ns` nanoseconds have passed, instead of
+// the system-dependent limit: a waiting warp then takes no issue slots from
+// the warps that share its SM sub-partition.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return done != 0;
+}
+
+#ifndef FA_WAIT_HINT_NS
+#define FA_WAIT_HINT_NS 0
+#endif
+
+// Non-blocking check that the phase with the given parity has completed.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
 // Status bits a kernel may raise in its device status word.
 enum : uint32_t {
   kStatusTimeout = 1u,  // a bounded wait gave up
@@ -74,7 +107,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(a, parity)) return true;
+    if (FA_WAIT_HINT_NS ? mbar_try_wait_sleep(a, parity, FA_WAIT_HINT_NS) : mbar_try_wait(a, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
       if (global_timer_ns() - t0 > timeout_ns) {
@@ -249,6 +282,18 @@ __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&a)[16], uint32_t (&
       : "memory");
 }
 
+// tcgen05.wait::ld that also names the 64 destination registers of two
+// 32-column loads, so that no use of them is scheduled before the wait even
+// when other work sits between the loads and the wait.
+__device__ __forceinline__ void tmem_wait_ld_regs32x2(uint32_t (&a)[32], uint32_t (&b)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7]), "+r"(a[8]), "+r"(a[9]), "+r"(a[10]), "+r"(a[11]), "+r"(a[12]), "+r"(a[13]), "+r"(a[14]), "+r"(a[15]), "+r"(a[16]), "+r"(a[17]), "+r"(a[18]), "+r"(a[19]), "+r"(a[20]), "+r"(a[21]), "+r"(a[22]), "+r"(a[23]), "+r"(a[24]), "+r"(a[25]), "+r"(a[26]), "+r"(a[27]), "+r"(a[28]), "+r"(a[29]), "+r"(a[30]), "+r"(a[31]),
+        "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]), "+r"(b[6]), "+r"(b[7]), "+r"(b[8]), "+r"(b[9]), "+r"(b[10]), "+r"(b[11]), "+r"(b[12]), "+r"(b[13]), "+r"(b[14]), "+r"(b[15]), "+r"(b[16]), "+r"(b[17]), "+r"(b[18]), "+r"(b[19]), "+r"(b[20]), "+r"(b[21]), "+r"(b[22]), "+r"(b[23]), "+r"(b[24]), "+r"(b[25]), "+r"(b[26]), "+r"(b[27]), "+r"(b[28]), "+r"(b[29]), "+r"(b[30]), "+r"(b[31])
+      :
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
@@ -379,21 +424,6 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   uint64_t d;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
   return bits_f2(d);
-}
-
-// Two floats to a bf16 pair (lo in bits 0-15) rounded to nearest, ties away
-// from zero, in integer arithmetic: adding half a unit of the last kept place
-// (0x8000) to each bit pattern carries into the kept 16 bits exactly when the
-// dropped 16 bits are at least half a unit, and one byte permute keeps the two
-// high halves.  It differs from round-to-nearest-even only on exact ties.
-// Infinities stay infinite and finite values past the largest bf16 become
-// infinite, as with round-to-nearest; NaN inputs give an undefined result.
-// On B200 this runs on the integer pipe.  The converting instruction
-// (cvt.rn.bf16x2.f32) applied to results of ex2.approx measured about 16
-// cycles per warp instruction in the softmax loop instead of 2, doubling the
-// loop's time, so the hot loops pack with this form.
-__device__ __forceinline__ uint32_t round_pack_bf16x2(float lo, float hi) {
-  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -114,6 +114,7 @@ def _stream_handle(stream) -> int:
 
 
 def _check_qkvo(q, k, v, o):
+    shape = q.shape
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
         if t.dtype != torch.bfloat16:
             raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
@@ -121,9 +122,11 @@ def _check_qkvo(q, k, v, o):
             raise ValueError(f"{name} must be a CUDA tensor")
         if not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
-        if t.dim() != 4:
-            raise ValueError(f"{name} must be [B, H, N, d]")
-    if not (q.shape == k.shape == v.shape == o.shape):
+        if t.shape != shape:
+            break
+    if len(shape) != 4:
+        raise ValueError("q must be [B, H, N, d]")
+    if not (shape == k.shape == v.shape == o.shape):
         raise ValueError(f"shape mismatch: q{tuple(q.shape)} k{tuple(k.shape)} "
                          f"v{tuple(v.shape)} o{tuple(o.shape)}")
 
@@ -137,6 +140,20 @@ def _lse_ptr(lse, B: int, H: int, N: int):
     if tuple(lse.shape) != (B, H, N):
         raise ValueError(f"lse must be [B, H, N] = {(B, H, N)}")
     return lse.data_ptr()
+
+
+def _launch_device_index(stream, first, *rest) -> int:
+    """Index of the one CUDA device all tensors (and the stream) live on.
+
+    The same check as _launch_device, on device indices: the cheaper form
+    for the per-call path of fa_fwd."""
+    dev = first.get_device()
+    for t in rest:
+        if t is not None and t.get_device() != dev:
+            raise ValueError("all tensors must be on one CUDA device")
+    if stream is not None and stream.device_index != dev:
+        raise ValueError(f"stream is on cuda:{stream.device_index}, tensors on cuda:{dev}")
+    return dev
 
 
 def _launch_device(stream, *tensors) -> torch.device:
@@ -163,16 +180,21 @@ def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
     scale: defaults to 1/sqrt(d).  Asynchronous on ``stream`` (default: the
     current stream of the tensors' device).
     """
-    lib = _load()
+    lib = _lib if _lib is not None else _load()
     _check_qkvo(q, k, v, o)
     B, H, N, d = q.shape
     lse_ptr = _lse_ptr(lse, B, H, N)
-    dev = _launch_device(stream, q, k, v, o, lse)
+    dev = _launch_device_index(stream, q, k, v, o, lse)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    with torch.cuda.device(dev):
-        _check(lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_ptr,
-                          B, H, N, d, float(scale), int(bool(causal)), _stream_handle(stream)))
+    handle = stream.cuda_stream if stream is not None else torch.cuda.current_stream(dev).cuda_stream
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_ptr, B, H, N, d, float(scale),
+            int(bool(causal)), handle)
+    if torch.cuda.current_device() == dev:
+        _check(lib.fa_fwd(*args))
+    else:
+        with torch.cuda.device(dev):
+            _check(lib.fa_fwd(*args))
 
 
 def fa_fwd_tile_config(q, k, v, o, lse=None, query_rows: int = 256, key_tile: int = 128,
