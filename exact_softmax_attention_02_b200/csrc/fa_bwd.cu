@@ -78,11 +78,14 @@ __device__ uint32_t g_bwd_status;
 constexpr int kTraceCtas = 16;
 constexpr int kTraceIters = 64;
 __device__ unsigned long long* g_bwd_trace;  // [2][kTraceCtas][4 roles][kTraceIters][8 events]
+// (the clock is read before the buffer's address is loaded, so that the load
+// cannot delay the stamp)
 #define BWD_TRACE(k, role, iter, ev)                                                                   \
   do {                                                                                                 \
-    if (g_bwd_trace != nullptr && blockIdx.x < kTraceCtas && (iter) < kTraceIters)                     \
+    const unsigned long long now_ = clock64();                                                         \
+    if (blockIdx.x < kTraceCtas && (iter) < kTraceIters && g_bwd_trace != nullptr)                     \
       g_bwd_trace[(((static_cast<size_t>(k) * kTraceCtas + blockIdx.x) * 4 + (role)) * kTraceIters +   \
-                   (iter)) * 8 + (ev)] = clock64();                                                     \
+                   (iter)) * 8 + (ev)] = now_;                                                          \
   } while (0)
 #else
 #define BWD_TRACE(k, role, iter, ev) \

@@ -128,13 +128,22 @@ __device__ __forceinline__ constexpr bool in_bounds(bool, uint32_t) { return tru
 constexpr int kTraceCtas = 16;
 constexpr int kTraceIters = 64;
 __device__ unsigned long long* g_trace;  // [kTraceCtas][4 roles][kTraceIters][8 events]
-#define FA_TRACE_MARK(role, iter, ev)                                                         \
-  do {                                                                                        \
-    if (g_trace != nullptr && blockIdx.x < kTraceCtas && (iter) < kTraceIters)                \
-      g_trace[((static_cast<size_t>(blockIdx.x) * 4 + (role)) * kTraceIters + (iter)) * 8 + \
-              (ev)] = clock64();                                                              \
+// The buffer's address is read once per thread at the start of the kernel
+// (FA_TRACE_INIT): a stamp is then a clock read and a store, with no load in
+// front of the clock that could delay it.
+#define FA_TRACE_INIT() unsigned long long* const trace_buf = blockIdx.x < kTraceCtas ? g_trace : nullptr
+#define FA_TRACE_MARK(role, iter, ev)                                                        \
+  do {                                                                                       \
+    if (trace_buf != nullptr && (iter) < kTraceIters) {                                      \
+      const unsigned long long now = clock64();                                              \
+      trace_buf[((static_cast<size_t>(blockIdx.x) * 4 + (role)) * kTraceIters + (iter)) * 8 + \
+                (ev)] = now;                                                                 \
+    }                                                                                        \
   } while (0)
 #else
+#define FA_TRACE_INIT() \
+  do {                  \
+  } while (0)
 #define FA_TRACE_MARK(role, iter, ev) \
   do {                                \
   } while (0)
@@ -192,6 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  FA_TRACE_INIT();
   const int split = SPLIT ? static_cast<int>(blockIdx.x % p.num_splits) : 0;
   const int unit = SPLIT ? static_cast<int>(blockIdx.x / p.num_splits) : static_cast<int>(blockIdx.x);
   // Work order: heads in groups of p.group_heads; inside a group, query
@@ -402,7 +412,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sv = iv % S, sk = ik % S;
         const bool last = it == n_iter - 1;
         if (!(ok = mbar_wait(&kv_full[sv], static_cast<uint32_t>(iv / S) & 1u, abort_flag, status, tmo, kSiteKvFull))) break;
-        bool k_ready = false;
+        FA_TRACE_MARK(3, it, 0);
+        // the next K tile too, here rather than between a PV and an S
+        // product: it has normally landed long before, but the wait itself
+        // costs the issuing thread time that the tensor core then idles
+        if (!last && !(ok = mbar_wait(&kv_full[sk], static_cast<uint32_t>(ik / S) & 1u, abort_flag, status, tmo,
+                                      kSiteKvFull)))
+          break;
+        FA_TRACE_MARK(3, it, 1);
         for (int t = 0; t < 2; ++t) {
           if (it >= first_it[t]) {
             const uint32_t ph = static_cast<uint32_t>(it - first_it[t]) & 1u;
@@ -415,10 +432,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (last) commit(&o_full[t]);
           }
           if (!last && it + 1 >= first_it[t]) {
-            if (!k_ready) {
-              if (!(ok = mbar_wait(&kv_full[sk], static_cast<uint32_t>(ik / S) & 1u, abort_flag, status, tmo, kSiteKvFull))) break;
-              k_ready = true;
-            }
             if (!q_ready[t]) {
               if (!(ok = mbar_wait(&q_full[t], 0, abort_flag, status, tmo, kSiteQ))) break;
               q_ready[t] = true;
