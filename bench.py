@@ -454,8 +454,6 @@ def run_ours(args, w):
         raise RuntimeError("kernel reported a device timeout during warm-up")
 
     sampler = ClockSampler(local_rank, period_s=float(os.environ.get("FA_BENCH_CLOCK_PERIOD", "0.01")))
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler.start()
     if dist is not None:
@@ -463,11 +461,11 @@ def run_ours(args, w):
     torch.cuda.synchronize(dev)
     if args.path == "standard":
         std_events = []
+    # the timed region: K steps between two events on the launching stream
+    # (no event between steps, so small problems are not charged for them)
     t_start.record(stream)
-    for i in range(args.steps):
-        ev[i][0].record(stream)
+    for _ in range(args.steps):
         step()
-        ev[i][1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize(dev)
     if dist is not None:
@@ -476,9 +474,23 @@ def run_ours(args, w):
     if fa.device_status(stream) != 0:
         raise RuntimeError("kernel reported a device timeout in the timed region")
     elapsed = t_start.elapsed_time(t_end) / 1e3
-    launch_ms = [a.elapsed_time(b) for a, b in ev]
     elapsed_max = max_over_ranks(elapsed, dist, dev)
-    avg_launch_s = max_over_ranks(sum(launch_ms) / len(launch_ms) / 1e3, dist, dev)
+    # device time per step over the timed region: the launches are queued
+    # back to back, so this is the average launch duration (all kernels of a
+    # step together when a step has several)
+    avg_launch_s = elapsed_max / args.steps
+    # the spread of single launches, from a separate untimed pass with an
+    # event pair around each step (the comparator's softmax events stay those
+    # of the timed region)
+    std_timed, std_events = std_events, None
+    n_spread = min(args.steps, 30)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_spread)]
+    for a, b in ev:
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
 
     # end to end through the public API: pinned host inputs -> device -> O, LSE back to host
     o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
@@ -548,7 +560,7 @@ def run_ours(args, w):
     if args.path == "standard":
         # the comparator's dominant kernel is the HBM-bound row softmax:
         # it reads the fp32 scores and writes the bf16 probabilities and LSE
-        sm_ms = [a.elapsed_time(b) for a, b in std_events]
+        sm_ms = [a.elapsed_time(b) for a, b in std_timed]
         sm_s = max_over_ranks(sum(sm_ms) / 1e3 / args.steps, dist, dev)
         nbytes = w.B * w.H * w.N * (6 * w.N + 4)
         hbm, hbm_src = hbm_peak()
@@ -559,7 +571,8 @@ def run_ours(args, w):
     launches = int(sum_over_ranks(args.steps * launches_per_step, dist, dev))
     srt = sorted(launch_ms)
     step_ms = {"min": srt[0], "median": srt[len(srt) // 2], "max": srt[-1],
-               "first5_mean": sum(launch_ms[:5]) / min(5, len(launch_ms))}
+               "first5_mean": sum(launch_ms[:5]) / min(5, len(launch_ms)),
+               "launches": len(launch_ms), "note": "single launches after the timed region"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and bwd is None:

@@ -431,6 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = mbar_wait(&ds_ready[qq], static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteDs)))
             break;
           if (qq == 0) BWD_TRACE(0, 0, it, 2);
+          BWD_TRACE(0, 0, it, 4 + qq);
           tc_fence_after();
           issue_acc_q(tmem + kColAcc, tmem + kColS, dO, qq, it > 0);      // dV += P^T dO
           issue_acc_q(tmem + kColAcc + D, tmem + kColDP, q, qq, it > 0);  // dK += dS^T Q
@@ -655,6 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = mbar_wait(&ds_ready[qq], static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteDs)))
             break;
           if (qq == 0) BWD_TRACE(1, 0, it, 2);
+          BWD_TRACE(1, 0, it, 4 + qq);
           tc_fence_after();
           // dQ += dS K: A = dS in TMEM (over dP), B = K tile as [keys][d] (MN-major)
 #pragma unroll
