@@ -13,8 +13,8 @@
 // fused tiled computation; interactiveml.org "FlashAttention saves the
 // matrix, not the quadratic work").
 //
-// CTA layout (384 threads, one CTA per SM):
-//   warp 0      TMA producer: Q tiles once, then K/V tiles through a ring of
+// CTA layout (384 threads, one persistent CTA per SM):
+//   warp 0      TMA producer: Q tiles, then K/V tiles through a ring of
 //               shared-memory stages guarded by full/empty mbarriers.
 //   warp 1      TMEM owner and MMA issuer (one thread): S_t = Q_t K^T
 //               (SS MMA, M=128 N=128 K=d) and O_t += P_t V (TS MMA, P from
@@ -22,8 +22,13 @@
 //   warps 2-3   idle.
 //   warps 4-7   softmax + epilogue for query tile 0 (one thread per row).
 //   warps 8-11  softmax + epilogue for query tile 1.
-// Each CTA owns 2 query tiles of 128 rows (256 rows of one head) so that the
-// softmax of one tile overlaps the MMAs of the other.
+// Warps 0-3 give registers up to the softmax warpgroups (setmaxnreg): 136
+// and 184 per thread (152 and 176 for d = 64 causal) against the 168 of the
+// launch.
+// A work item is 2 query tiles of 128 rows (256 rows of one head) so that the
+// softmax of one tile overlaps the MMAs of the other.  Each CTA takes items
+// gridDim.x apart until none is left; the next item's loads and first score
+// products overlap the previous item's last products and epilogue.
 //
 // Tensor memory (512 columns x 128 lanes of 32 bit):
 //   [0,128)      S_0, fp32; P_0 (bf16 pairs) overwrites its first 64 columns
@@ -68,12 +73,25 @@ static_assert(FA_BLOCK_Q == kQTiles * kBM && FA_BLOCK_K == kBN,
               "a block-sparse block is one CTA's query rows by one key tile");
 constexpr int kThreads = 384;  // 12 warps
 constexpr int kSoftmaxWarp0 = 4;
+// Registers per thread after the split between warpgroup 0 (producer, MMA,
+// two idle warps) and the two softmax warpgroups, with 128 * control + 256 *
+// softmax = 384 * 168, the 64K register file at the launch's 168 per thread:
+// the smallest control share that compiles without spills (found with
+// -Xptxas -v), the rest to the softmax.
+template <int D, bool CAUSAL, bool SPLIT, bool SPARSE>
+__host__ __device__ constexpr uint32_t regs_control() {
+  return (D == 64 && CAUSAL && !SPLIT && !SPARSE) ? 152 : 136;
+}
+template <int D, bool CAUSAL, bool SPLIT, bool SPARSE>
+__host__ __device__ constexpr uint32_t regs_softmax() {
+  return (kThreads * 168 - 128 * regs_control<D, CAUSAL, SPLIT, SPARSE>()) / 256;
+}
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr uint32_t kTmemCols = 512;
 // wait sites reported in the device status word (bit 8 + site)
 enum : uint32_t {
   kSiteKvEmpty = 0, kSiteQ = 1, kSiteKvFull = 2, kSiteS = 3, kSiteP = 4,  // 4..5: p_full[0..1]
-  kSiteO = 8, kSiteDebug = 9,
+  kSiteQFree = 6, kSiteSched = 7, kSiteO = 8, kSiteDebug = 9,
 };
 constexpr int kChunkBytes = kBM * 64 * 2;  // one 64-wide, 128-row swizzled box: 16 KB
 
@@ -153,19 +171,102 @@ template <int D, int BN = kBN>
 struct Cfg {
   static_assert(BN == 128 || BN == 64, "key tiles of 128 or 64");
   static constexpr int kChunks = D / 64;
-  static constexpr int kQBytes = kBM * D * 2;  // one query tile (reused as O staging)
+  static constexpr int kQBytes = kBM * D * 2;  // one query tile
   static constexpr int kStageBytes = BN * D * 2;  // one ring stage: a whole K or V tile
   static constexpr int kKChunkBytes = BN * 128;   // one 64-wide d chunk of a K stage
   static constexpr int kVChunkBytes = BN * 128;   // one 64-wide d chunk of a V stage
   // the same ring bytes whatever the tile: more stages for smaller tiles
   static constexpr int kStages = (D == 64 ? 8 : 4) * (128 / BN);
-  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 1 + 1;
-  static constexpr int kSmemTiles = kQTiles * kQBytes + kStages * kStageBytes;
-  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 1024;
+  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 2 + 1 + 1 + 2 + 2 + 1;
+  // O staging: one 32-row x 64-column bf16 box (128-byte rows) per softmax warp
+  static constexpr int kOStageBytes = 32 * 128;
+  static constexpr int kSmemTiles = kQTiles * kQBytes + kStages * kStageBytes + 8 * kOStageBytes;
+  // control block: launch-cancel answer (16 B), barriers, next-item slots,
+  // TMEM base and abort flag (16 B), and the slack for 1024-byte alignment
+  static constexpr int kSmemBytes = kSmemTiles + 16 + kNumBars * 8 + 16 + 1024;
   static constexpr uint32_t kColO = 256;
 };
 
-// One CTA owns two 128-row query tiles of one head and issues M=128 MMAs.
+// The work of one unit: a 256-row query block (two 128-row tiles, or one
+// for the tile-size sweep) of one head, and for split-KV one key range.
+struct Unit {
+  int bh, qblk, split, q0;
+  int j_last[2];
+  int kv_lo, kv_end, n_iter;
+  int first_it[2];
+  bool active[2];
+  const int* blk;  // block-sparse: this block's retained key tiles
+};
+
+// Work item w, in heavy-first order: heads in groups of p.group_heads;
+// inside a group, query blocks from the heaviest (last rows: most keys when
+// causal) to the lightest, cycling over the group's heads, so that blocks
+// running together share the K/V of a few heads in L2; split-KV ranges of one
+// block are adjacent.
+template <bool CAUSAL, bool SPLIT, bool SPARSE, int BN, int QT>
+__device__ __forceinline__ Unit unit_of(const FwdParams& p, int w) {
+  Unit u;
+  u.split = SPLIT ? w % p.num_splits : 0;
+  const int unit = SPLIT ? w / p.num_splits : w;
+  const int per_group = p.group_heads * p.n_qblk;
+  const int grp = unit / per_group;
+  const int rem = unit % per_group;
+  const int grp_heads = min(p.group_heads, p.BH - grp * p.group_heads);
+  u.bh = grp * p.group_heads + rem % grp_heads;
+  u.qblk = p.n_qblk - 1 - rem / grp_heads;
+  u.q0 = u.qblk * QT * kBM - (2 - QT) * kBM;  // first row of slot 0
+  // last key tile each query tile needs (the causal diagonal, or the end)
+#pragma unroll
+  for (int t = 0; t < 2; ++t)
+    u.j_last[t] = CAUSAL ? min(u.q0 + (t + 1) * kBM - 1, p.N - 1) / BN : p.n_kv - 1;
+  // key tiles [kv_lo, kv_end) of this unit (all of them unless split),
+  // visited from kv_end - 1 down to kv_lo
+  u.kv_lo = SPLIT ? u.split * p.kv_per_split : 0;
+  u.kv_end = SPLIT ? min(u.j_last[1] + 1, u.kv_lo + p.kv_per_split) : u.j_last[1] + 1;
+  u.n_iter = max(0, u.kv_end - u.kv_lo);
+  // iterations before a query tile's first unmasked key tile are skipped for
+  // it; a tile whose first iteration is past n_iter has no keys in this range
+  u.first_it[0] = u.kv_end - 1 - min(u.j_last[0], u.kv_end - 1);
+  u.first_it[1] = 0;
+  u.blk = nullptr;
+  // Block-sparse: this block's retained key tiles, visited from the last
+  // entry down.  Entries past tile 1's diagonal are seen by no row and are
+  // dropped; leading visits past tile 0's diagonal are skipped for tile 0.
+  // A malformed list raises kStatusLayout; out-of-range or out-of-order
+  // entries are then masked out entirely (no memory outside the tensors is
+  // touched), and the outputs are not meaningful.
+  if (SPARSE) {
+    int beg = __ldg(p.blk_row_ptr + u.qblk), end = __ldg(p.blk_row_ptr + u.qblk + 1);
+    if (!(0 <= beg && beg <= end && end <= p.blk_nnz)) {
+      if (threadIdx.x == 0) atomicOr(&g_device_status, kStatusLayout);
+      beg = end = 0;
+    }
+    u.blk = p.blk_col_idx + beg;
+    int n = end - beg;
+    while (n > 0 && __ldg(u.blk + n - 1) > u.j_last[1]) {
+      if (threadIdx.x == 0 && __ldg(u.blk + n - 1) >= p.n_kv) atomicOr(&g_device_status, kStatusLayout);
+      --n;
+    }
+    int skip = 0;
+    while (skip < n && __ldg(u.blk + n - 1 - skip) > u.j_last[0]) ++skip;
+    u.n_iter = n;
+    u.first_it[0] = skip;
+  }
+  if (QT == 1) u.first_it[0] = u.n_iter;  // slot 0 unused
+  u.active[0] = u.first_it[0] < u.n_iter;
+  u.active[1] = u.n_iter > 0;
+  return u;
+}
+
+// One CTA is launched per work item, in heavy-first order, but a CTA does
+// not end with its item: its producer thread asks the hardware to cancel the
+// launch of the next pending CTA (cluster launch control) and takes that
+// CTA's item over, until none is left.  The SMs so take the items in launch
+// order, as free SMs would take new CTAs (greedy longest-first), while each
+// CTA keeps its tensor memory, barriers and pipeline: every barrier counts
+// its phases on from one item to the next, and the next item's Q and K/V
+// tiles load, and its first score products run, while the previous item's
+// last products and epilogue finish.
 template <int D, bool CAUSAL, bool SPLIT, bool SPARSE, int BN, int QT>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -184,86 +285,41 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem;                  // kQTiles query tiles (reused as O staging)
+  uint8_t* sQ = smem;                  // kQTiles query tiles
   uint8_t* sKV = smem + kQTiles * QB;  // S ring stages
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemTiles);
+  uint8_t* sO = sKV + S * SB;          // O staging, one box per softmax warp
+  uint8_t* ctrl = smem + C::kSmemTiles;
+  void* clc_resp = ctrl;              // 16 B: answer of the last launch-cancel request
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ctrl + 16);
   uint64_t* q_full = bars;            // [2] Q tile landed
   uint64_t* kv_full = q_full + 2;     // [S] K/V stage landed
   uint64_t* kv_empty = kv_full + S;   // [S] MMA -> producer
   uint64_t* s_full = kv_empty + S;    // [2] MMA -> softmax
   uint64_t* p_full = s_full + 2;      // [2] softmax -> MMA
   uint64_t* o_full = p_full + 2;      // [2] MMA -> epilogue
-  uint64_t* mma_done = o_full + 2;    // [1] MMA -> itself, before TMEM release
+  uint64_t* q_free = o_full + 2;      // [2] MMA -> producer: an item's last S product of tile t is done
+  uint64_t* mma_done = q_free + 2;    // [1] MMA -> itself, before TMEM release
   uint64_t* never = mma_done + 1;     // [1] debug: nothing arrives here
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
+  uint64_t* sched_full = never + 1;   // [2] producer -> MMA, softmax: next item id written
+  uint64_t* sched_empty = sched_full + 2;  // [2] MMA, softmax -> producer: id read
+  uint64_t* clc_bar = sched_empty + 2;     // [1] launch-cancel answer landed
+  volatile int* sched_item = reinterpret_cast<volatile int*>(clc_bar + 1);  // [2] next item, -1: none
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(sched_item) + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* status = &g_device_status;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   FA_TRACE_INIT();
-  const int split = SPLIT ? static_cast<int>(blockIdx.x % p.num_splits) : 0;
-  const int unit = SPLIT ? static_cast<int>(blockIdx.x / p.num_splits) : static_cast<int>(blockIdx.x);
-  // Work order: heads in groups of p.group_heads; inside a group, query
-  // blocks from the heaviest (last rows: most keys when causal) to the
-  // lightest, cycling over the group's heads.  Blocks that run together then
-  // share the K/V of a few heads in L2, and light blocks end the grid.
-  const int per_group = p.group_heads * p.n_qblk;
-  const int grp = unit / per_group;
-  const int rem = unit % per_group;
-  const int grp_heads = min(p.group_heads, p.BH - grp * p.group_heads);
-  const int bh = grp * p.group_heads + rem % grp_heads;
-  const int qblk = p.n_qblk - 1 - rem / grp_heads;
-  const int q0 = qblk * QT * kBM - (2 - QT) * kBM;  // first row of slot 0
-  // last key tile each query tile needs (the causal diagonal, or the end)
-  int j_last[2];
-#pragma unroll
-  for (int t = 0; t < 2; ++t)
-    j_last[t] = CAUSAL ? min(q0 + (t + 1) * kBM - 1, p.N - 1) / BN : p.n_kv - 1;
-  // key tiles [kv_lo, kv_end) of this CTA (all of them unless split), visited
-  // from kv_end-1 down to kv_lo
-  const int kv_lo = SPLIT ? split * p.kv_per_split : 0;
-  const int kv_end = SPLIT ? min(j_last[1] + 1, kv_lo + p.kv_per_split) : j_last[1] + 1;
-  int n_iter = max(0, kv_end - kv_lo);
-  // iterations before a query tile's first unmasked key tile are skipped for
-  // it; a tile whose first iteration is past n_iter has no keys in this range
-  int first_it[2] = {kv_end - 1 - min(j_last[0], kv_end - 1), 0};
-  // Block-sparse: this block's retained key tiles, visited from the last
-  // entry down.  Entries past tile 1's diagonal are seen by no row and are
-  // dropped; leading visits past tile 0's diagonal are skipped for tile 0.
-  // A malformed list raises kStatusLayout; out-of-range or out-of-order
-  // entries are then masked out entirely (no memory outside the tensors is
-  // touched), and the outputs are not meaningful.
-  const int* blk = nullptr;
-  if (SPARSE) {
-    int beg = __ldg(p.blk_row_ptr + qblk), end = __ldg(p.blk_row_ptr + qblk + 1);
-    if (!(0 <= beg && beg <= end && end <= p.blk_nnz)) {
-      if (threadIdx.x == 0) atomicOr(&g_device_status, kStatusLayout);
-      beg = end = 0;
-    }
-    blk = p.blk_col_idx + beg;
-    int n = end - beg;
-    while (n > 0 && __ldg(blk + n - 1) > j_last[1]) {
-      if (threadIdx.x == 0 && __ldg(blk + n - 1) >= p.n_kv) atomicOr(&g_device_status, kStatusLayout);
-      --n;
-    }
-    int skip = 0;
-    while (skip < n && __ldg(blk + n - 1 - skip) > j_last[0]) ++skip;
-    n_iter = n;
-    first_it[0] = skip;
-  }
-  if (QT == 1) first_it[0] = n_iter;  // slot 0 unused
-  const bool tile_active[2] = {first_it[0] < n_iter, n_iter > 0};
-  // key tile of iteration it
-  auto kv_tile = [&](int it) { return SPARSE ? __ldg(blk + n_iter - 1 - it) : kv_end - 1 - it; };
   const uint64_t tmo = p.timeout_ns;
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
       mbar_init(&q_full[t], 1);
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], kBM);
+      mbar_init(&p_full[t], kBM / 32);  // one arrival per softmax warp
       mbar_init(&o_full[t], 1);
+      mbar_init(&q_free[t], 1);
     }
     for (int s = 0; s < S; ++s) {
       mbar_init(&kv_full[s], 1);
@@ -271,12 +327,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(mma_done, 1);
     mbar_init(never, 1);
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&sched_full[k], 1);
+      // the MMA thread and every softmax warp read each id
+      mbar_init(&sched_empty[k], 1 + (kBM / 32) * QT);
+    }
+    mbar_init(clc_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
-    tma_prefetch_desc(&tmO);
+    if (!SPLIT) tma_prefetch_desc(&tmO);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -289,58 +351,105 @@ __global__ void __launch_bounds__(kThreads, 1)
   static_assert(2 * BN <= C::kColO && C::kColO + 2 * D <= kTmemCols, "S_0, S_1, O_0, O_1 fit the allocation");
   // (all 512 columns are allocated, so the base column is 0)
   if (threadIdx.x == 0) in_bounds((tmem & 0xffffu) == 0, kCheckTmem);
-
-  // rows of this CTA's query tile t
-  auto tile_row0 = [&](int t) { return q0 + t * kBM; };
-
+  // Every warp, converged, inside its role's branch (so that the role's code
+  // is compiled for its count): warpgroup 0 gives registers up, the softmax
+  // warpgroups take them.
+  constexpr uint32_t kRegsControl = regs_control<D, CAUSAL, SPLIT, SPARSE>();
+  constexpr uint32_t kRegsSoftmax = regs_softmax<D, CAUSAL, SPLIT, SPARSE>();
+  static_assert(kRegsControl % 8 == 0 && kRegsSoftmax % 8 == 0 &&
+                    128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * 168,
+                "the split fits the launch's registers");
+  if (warp < kSoftmaxWarp0) regs_dealloc<kRegsControl>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && n_iter > 0) {
+    if (lane == 0) {
       bool ok = true;
-      bool q_issued[2] = {false, false};
-      if (tile_active[0]) {
-        if (in_bounds(tile_row0(0) >= 0 && tile_row0(0) < p.n_qblk * QT * kBM && bh < p.BH, kCheckQLoad)) {
-          q_issued[0] = true;
-          mbar_arrive_expect_tx(&q_full[0], QB);
-          for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(sQ + c * kChunkBytes, &tmQ, &q_full[0], c * 64, tile_row0(0), bh);
-        } else {
-          ok = false;
-          *abort_flag = 1;
+      int i = 0;                     // loads issued into the ring, over all items
+      int q_loads[2] = {0, 0};       // loads issued into each Q buffer
+      bool clc_open = true;          // launches may be left to take over
+      bool clc_pending = false;      // a request whose answer is not read yet
+      uint32_t clc_phase = 0;
+      int w = static_cast<int>(blockIdx.x);
+      // Asks for the next item.  Asked at the start of this item's last
+      // loads, about two iterations before the CTA finishes it (the loads
+      // run that far ahead of the products), so that items go to CTAs in the
+      // order in which they finish, as with new CTAs on free SMs; asked at
+      // the start of an item, the second round of items would be dealt out
+      // before any CTA is near its end (measured: 10% slower on causal
+      // N = 8192).  The answer is read once the item's loads are issued.
+      auto request_next = [&]() {
+        if (clc_open && !clc_pending) {
+          mbar_arrive_expect_tx(clc_bar, 16);
+          clc_try_cancel(clc_resp, clc_bar);
+          clc_pending = true;
         }
-      }
-      int i = 0;  // loads issued into the ring, in consumption order K0 V0 K1 V1 ...
-      for (int it = 0; it < n_iter && ok; ++it) {
-        // (a block-sparse entry out of range is loaded clamped and masked)
-        const int j = SPARSE ? min(max(kv_tile(it), 0), p.n_kv - 1) : kv_tile(it);
-        for (int kv = 0; kv < 2; ++kv) {
-          const int s = i % S;
-          const uint32_t ph = static_cast<uint32_t>(i / S) & 1u;
-          ok = mbar_wait(&kv_empty[s], ph ^ 1u, abort_flag, status, tmo, kSiteKvEmpty);
-          if (!ok) break;
-          if (!in_bounds(j >= 0 && j < p.n_kv && s < S && bh < p.BH, kCheckKvLoad)) {
-            ok = false;
+      };
+      for (int k = 0; ok; ++k) {
+        const Unit u = unit_of<CAUSAL, SPLIT, SPARSE, BN, QT>(p, w);
+        // Q tile t of this item, once the previous item's last S product of
+        // tile t (the last reader of the buffer) has finished
+        auto load_q = [&](int t) {
+          if (q_loads[t] > 0 &&
+              !mbar_wait(&q_free[t], static_cast<uint32_t>(q_loads[t] - 1) & 1u, abort_flag, status, tmo, kSiteQFree))
+            return false;
+          const int row0 = u.q0 + t * kBM;
+          if (!in_bounds(row0 >= 0 && row0 < p.n_qblk * QT * kBM && u.bh < p.BH, kCheckQLoad)) {
             *abort_flag = 1;
-            break;
+            return false;
           }
-          mbar_arrive_expect_tx(&kv_full[s], SB);
-          uint8_t* st = sKV + s * SB;
-          const CUtensorMap* map = kv == 0 ? &tmK : &tmV;
-          for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(st + c * C::kKChunkBytes, map, &kv_full[s], c * 64, j * BN, bh);
-          ++i;
-          if (it == 0 && kv == 0) {
-            if (!in_bounds(tile_row0(1) >= 0 && tile_row0(1) < p.n_qblk * QT * kBM, kCheckQLoad)) {
+          ++q_loads[t];
+          mbar_arrive_expect_tx(&q_full[t], QB);
+          for (int ch = 0; ch < C::kChunks; ++ch)
+            tma_load_3d(sQ + t * QB + ch * kChunkBytes, &tmQ, &q_full[t], ch * 64, row0, u.bh);
+          return true;
+        };
+        if (u.active[0] && !(ok = load_q(0))) break;
+        // loads of this item in consumption order K0 V0 K1 V1 ... (none
+        // when the item has no key tile)
+        for (int it = 0; it < u.n_iter && ok; ++it) {
+          if (it == u.n_iter - 1) request_next();
+          // (a block-sparse entry out of range is loaded clamped and masked)
+          const int j = SPARSE ? min(max(__ldg(u.blk + u.n_iter - 1 - it), 0), p.n_kv - 1) : u.kv_end - 1 - it;
+          for (int kv = 0; kv < 2; ++kv) {
+            const int s = i % S;
+            const uint32_t ph = static_cast<uint32_t>(i / S) & 1u;
+            ok = mbar_wait(&kv_empty[s], ph ^ 1u, abort_flag, status, tmo, kSiteKvEmpty);
+            if (!ok) break;
+            if (!in_bounds(j >= 0 && j < p.n_kv && s < S && u.bh < p.BH, kCheckKvLoad)) {
               ok = false;
               *abort_flag = 1;
               break;
             }
-            q_issued[1] = true;
-            mbar_arrive_expect_tx(&q_full[1], QB);
-            for (int c = 0; c < C::kChunks; ++c)
-              tma_load_3d(sQ + QB + c * kChunkBytes, &tmQ, &q_full[1], c * 64, tile_row0(1), bh);
+            mbar_arrive_expect_tx(&kv_full[s], SB);
+            uint8_t* st = sKV + s * SB;
+            const CUtensorMap* map = kv == 0 ? &tmK : &tmV;
+            for (int ch = 0; ch < C::kChunks; ++ch)
+              tma_load_3d(st + ch * C::kKChunkBytes, map, &kv_full[s], ch * 64, j * BN, u.bh);
+            ++i;
+            if (it == 0 && kv == 0 && !(ok = load_q(1))) break;
           }
         }
+        if (!ok) break;
+        request_next();  // (an item without key tiles)
+        int next = -1;
+        if (clc_pending) {
+          if (!(ok = mbar_wait(clc_bar, clc_phase, abort_flag, status, tmo, kSiteSched))) break;
+          clc_phase ^= 1u;
+          clc_pending = false;
+          uint32_t x;
+          if (clc_query(clc_resp, &x))
+            next = static_cast<int>(x);
+          else
+            clc_open = false;  // no launch left: no further request may be made
+        }
+        // hand the next item (or the end, -1) to the MMA and softmax roles
+        if (!(ok = mbar_wait(&sched_empty[k & 1], (static_cast<uint32_t>(k >> 1) & 1u) ^ 1u, abort_flag, status,
+                             tmo, kSiteSched)))
+          break;
+        sched_item[k & 1] = next;
+        mbar_arrive(&sched_full[k & 1]);
+        if (next < 0) break;
+        w = next;
       }
       if (!ok) {
         // Unwinding: wait for every copy this CTA issued, so that none lands
@@ -350,12 +459,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait_drain(&kv_full[s], static_cast<uint32_t>(last / S) & 1u, tmo);
         }
         for (int t = 0; t < 2; ++t)
-          if (q_issued[t]) mbar_wait_drain(&q_full[t], 0, tmo);
+          if (q_loads[t] > 0) mbar_wait_drain(&q_full[t], static_cast<uint32_t>(q_loads[t] - 1) & 1u, tmo);
+        // and for the answer of a launch-cancel request still on its way
+        if (clc_pending) mbar_wait_drain(clc_bar, clc_phase, tmo);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_iter > 0) {
+    if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(kBM, BN, false);
       constexpr uint32_t idO = idesc_bf16_f32(kBM, D, true);
       const uint32_t sq = smem_addr(sQ);
@@ -394,279 +505,362 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(tmem + C::kColO + t * D, tmem + t * BN + kk * 8, bd, idO, acc);
         }
       };
-      auto commit = [&](uint64_t* bar) { mma_commit(bar); };
-      bool ok = mbar_wait(&kv_full[0], 0, abort_flag, status, tmo, kSiteKvFull);
-      bool q_ready[2] = {false, false};
-      for (int t = 0; t < 2 && ok; ++t) {
-        if (first_it[t] != 0) continue;
-        ok = mbar_wait(&q_full[t], 0, abort_flag, status, tmo, kSiteQ);
-        if (!ok) break;
-        q_ready[t] = true;
-        tc_fence_after();
-        issue_s(t, 0);
-        commit(&s_full[t]);
-      }
-      if (ok) commit(&kv_empty[0]);
-      for (int it = 0; it < n_iter && ok; ++it) {
-        const int iv = 2 * it + 1, ik = 2 * it + 2;
-        const int sv = iv % S, sk = ik % S;
-        const bool last = it == n_iter - 1;
-        if (!(ok = mbar_wait(&kv_full[sv], static_cast<uint32_t>(iv / S) & 1u, abort_flag, status, tmo, kSiteKvFull))) break;
-        FA_TRACE_MARK(3, it, 0);
-        // the next K tile too, here rather than between a PV and an S
-        // product: it has normally landed long before, but the wait itself
-        // costs the issuing thread time that the tensor core then idles
-        if (!last && !(ok = mbar_wait(&kv_full[sk], static_cast<uint32_t>(ik / S) & 1u, abort_flag, status, tmo,
-                                      kSiteKvFull)))
-          break;
-        FA_TRACE_MARK(3, it, 1);
-        for (int t = 0; t < 2; ++t) {
-          if (it >= first_it[t]) {
-            const uint32_t ph = static_cast<uint32_t>(it - first_it[t]) & 1u;
-            const bool acc = it > first_it[t];
-            if (!(ok = mbar_wait(&p_full[t], ph, abort_flag, status, tmo, kSiteP + t))) break;
-            FA_TRACE_MARK(0, it, 3 * t);
+      bool ok = true;
+      int i = 0;                     // ring loads consumed, over all items
+      int q_seen[2] = {0, 0};        // Q loads consumed per buffer
+      int p_seen[2] = {0, 0};        // P publications consumed per tile
+      int trace_it = 0;              // iterations over all items (trace stamps)
+      int w = static_cast<int>(blockIdx.x);
+      for (int k = 0; ok; ++k) {
+        const Unit u = unit_of<CAUSAL, SPLIT, SPARSE, BN, QT>(p, w);
+        const int n_iter = u.n_iter;
+        if (n_iter > 0) {
+          // the ring stage of load number n, waited for
+          auto wait_load = [&](int n) {
+            return mbar_wait(&kv_full[n % S], static_cast<uint32_t>(n / S) & 1u, abort_flag, status, tmo, kSiteKvFull);
+          };
+          auto wait_q = [&](int t) {
+            if (!mbar_wait(&q_full[t], static_cast<uint32_t>(q_seen[t]) & 1u, abort_flag, status, tmo, kSiteQ))
+              return false;
+            ++q_seen[t];
+            return true;
+          };
+          const int i0 = i;  // this item's first load: K0 at i0, V0 at i0 + 1, K1 at i0 + 2, ...
+          bool q_ready[2] = {false, false};
+          if (!(ok = wait_load(i0))) break;
+  #pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (!ok || u.first_it[t] != 0) continue;
+            if (!(ok = wait_q(t))) break;
+            q_ready[t] = true;
             tc_fence_after();
-            issue_pv(t, sv, acc);
-            FA_TRACE_MARK(0, it, 3 * t + 1);
-            if (last) commit(&o_full[t]);
+            issue_s(t, i0 % S);
+            mma_commit(&s_full[t]);
+            if (n_iter == 1) mma_commit(&q_free[t]);  // the item's last S product of tile t
           }
-          if (!last && it + 1 >= first_it[t]) {
-            if (!q_ready[t]) {
-              if (!(ok = mbar_wait(&q_full[t], 0, abort_flag, status, tmo, kSiteQ))) break;
-              q_ready[t] = true;
+          if (!ok) break;
+          mma_commit(&kv_empty[i0 % S]);
+          for (int it = 0; it < n_iter && ok; ++it) {
+            const int iv = i0 + 2 * it + 1, ik = i0 + 2 * it + 2;
+            const int sv = iv % S, sk = ik % S;
+            const bool last = it == n_iter - 1;
+            if (!(ok = wait_load(iv))) break;
+            FA_TRACE_MARK(3, trace_it + it, 0);
+            // the next K tile too, here rather than between a PV and an S
+            // product: it has normally landed long before, but the wait itself
+            // costs the issuing thread time that the tensor core then idles
+            if (!last && !(ok = wait_load(ik))) break;
+            FA_TRACE_MARK(3, trace_it + it, 1);
+  #pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              if (!ok) continue;
+              if (it >= u.first_it[t]) {
+                // (the first PV of an item overwrites O_t; the softmax threads
+                // that publish its P have read the previous item's O_t out
+                // of TMEM before, in their epilogue)
+                if (!(ok = mbar_wait(&p_full[t], static_cast<uint32_t>(p_seen[t]) & 1u, abort_flag, status, tmo,
+                                     kSiteP + t)))
+                  break;
+                ++p_seen[t];
+                FA_TRACE_MARK(0, trace_it + it, 3 * t);
+                tc_fence_after();
+                issue_pv(t, sv, it > u.first_it[t]);
+                FA_TRACE_MARK(0, trace_it + it, 3 * t + 1);
+                if (last) mma_commit(&o_full[t]);
+              }
+              if (!last && it + 1 >= u.first_it[t]) {
+                if (!q_ready[t]) {
+                  if (!(ok = wait_q(t))) break;
+                  q_ready[t] = true;
+                }
+                tc_fence_after();
+                issue_s(t, sk);
+                mma_commit(&s_full[t]);
+                if (it + 1 == n_iter - 1) mma_commit(&q_free[t]);  // the item's last S product of tile t
+                FA_TRACE_MARK(0, trace_it + it, 3 * t + 2);
+              }
             }
-            tc_fence_after();
-            issue_s(t, sk);
-            commit(&s_full[t]);
-            FA_TRACE_MARK(0, it, 3 * t + 2);
+            if (!ok) break;
+            mma_commit(&kv_empty[sv]);
+            if (!last) mma_commit(&kv_empty[sk]);
           }
+          i = i0 + 2 * n_iter;
+          trace_it += n_iter;
         }
         if (!ok) break;
-        commit(&kv_empty[sv]);
-        if (!last) commit(&kv_empty[sk]);
+        // the next item
+        if (!(ok = mbar_wait(&sched_full[k & 1], static_cast<uint32_t>(k >> 1) & 1u, abort_flag, status, tmo,
+                             kSiteSched)))
+          break;
+        const int next = sched_item[k & 1];
+        mbar_arrive(&sched_empty[k & 1]);
+        if (next < 0) break;
+        w = next;
       }
       // every MMA issued here has finished before TMEM is released
       mma_commit(mma_done);
       mbar_wait_drain(mma_done, 0, tmo);
     }
-  } else if (warp >= kSoftmaxWarp0 && (QT == 2 || warp >= kSoftmaxWarp0 + 4)) {
-    // ------------------------------------------------------------ softmax
-    const int t = (warp - kSoftmaxWarp0) >> 2;  // query tile of this warpgroup
-    const int wq = warp & 3;                    // TMEM lane quarter
-    const int r = wq * 32 + lane;               // row inside the tile
-    const int row0 = tile_row0(t);
-    const int row = row0 + r;                   // query index in the head
-    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_base + t * BN;
-    const uint32_t tO = tmem + lane_base + C::kColO + t * D;
-    const float sl2 = p.scale_log2;
-    // last key this row may see
-    const int key_limit = CAUSAL ? min(row, p.N - 1) : p.N - 1;
-    // O_t holds the product through the previous tile (that MMA finished
-    // before S_t of this tile was committed): rescale this thread's row of
-    // it in place, before P of this tile releases the next PV product.
-    auto rescale_o_rows = [&](uint32_t taddr, float a) {
-#pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
-        uint32_t o[16];
-        tmem_ld16(taddr + c * 16, o);
-        tmem_wait_ld();
-#pragma unroll
-        for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * a);
-        tmem_st16(taddr + c * 16, o);
-      }
-    };
-
-    float m_ref = -INFINITY;  // reference maximum, log2 units of scaled scores
-    float l_sum = 0.f;        // running denominator relative to m_ref
-    bool ok = true;
-    if (p.debug & 1u) {
-      ok = __all_sync(0xffffffffu, mbar_wait(never, 0, abort_flag, status, tmo, kSiteDebug));
-    }
-    for (int it = first_it[t]; it < n_iter && ok; ++it) {
-      const int li = it - first_it[t];
-      int j = kv_tile(it);
-      // a block-sparse entry out of range or out of order contributes nothing
-      bool bad = false;
-      if (SPARSE) {
-        bad = j < 0 || j >= p.n_kv || (it > 0 && j >= kv_tile(it - 1));
-        if (bad) {
-          if ((threadIdx.x & 127) == 0) atomicOr(&g_device_status, kStatusLayout);
-          j = 0;
-        }
-      }
-      ok = __all_sync(0xffffffffu,
-                      mbar_wait(&s_full[t], static_cast<uint32_t>(li) & 1u, abort_flag, status, tmo, kSiteS));
-      if (!ok) break;
-      const bool tr = lane == 0 && (warp & 3) == 0;
-      if (tr) FA_TRACE_MARK(1 + t, it, 0);
-      tc_fence_after();
-      constexpr int kQ32 = BN / 32;  // 32-key groups of a tile
-      uint32_t sr[kQ32][32];
-#pragma unroll
-      for (int q = 0; q < kQ32; ++q) tmem_ld32(tS + q * 32, sr[q]);
-      tmem_wait_ld();
-      if (tr) FA_TRACE_MARK(1 + t, it, 1);
-
-      const int kbase = j * BN;
-      const bool masked = bad || (kbase + BN > p.N) || (CAUSAL && kbase + BN - 1 > row0);
-      if (masked) {
-        const int lim = bad ? -1 : key_limit;
-#pragma unroll
-        for (int q = 0; q < kQ32; ++q)
-#pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (kbase + q * 32 + c > lim) sr[q][c] = __float_as_uint(-INFINITY);
-      }
-      // row maximum of the raw scores (scale > 0 keeps the argmax): BN/16
-      // independent chains of three-input maxima
-      constexpr int kChains = BN / 16;
-      float mx[kChains];
-#pragma unroll
-      for (int k = 0; k < kChains; ++k) mx[k] = __uint_as_float(sr[k >> 1][(k & 1) * 16]);
-#pragma unroll
-      for (int k = 0; k < kChains; ++k) {
-        const uint32_t* v = &sr[k >> 1][(k & 1) * 16];
-#pragma unroll
-        for (int c = 1; c < 15; c += 2)
-          mx[k] = fmax3(mx[k], __uint_as_float(v[c]), __uint_as_float(v[c + 1]));
-        mx[k] = fmaxf(mx[k], __uint_as_float(v[15]));
-      }
-      float m_all;
-      if constexpr (kChains == 8)
-        m_all = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-      else
-        m_all = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]);
-      const float m_tile = m_all * sl2;
-      if (tr) FA_TRACE_MARK(1 + t, it, 2);
-      // raise the reference maximum only when this tile exceeds it by > 2^8
-      const bool raise = m_tile > m_ref + kRescaleThreshold;
-      float alpha = 1.f;
-      if (raise) {
-        alpha = ex2_approx(m_ref - m_tile);  // 0 while m_ref is -inf
-        m_ref = m_tile;
-      }
-      const bool rescale_o = li > 0 && __any_sync(0xffffffffu, raise);
-      const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-      const float2 sl2v = make_float2(sl2, sl2);
-      const float2 nm2 = make_float2(neg_m, neg_m);
-      float2 ps2[kQ32];
-      // p = 2^(s * scale * log2 e - m), written as bf16 pairs over the first
-      // BN/2 columns of S_t, 64 keys at a time, and published whole on
-      // p_full[t].
-#pragma unroll
-      for (int h = 0; h < BN / 64; ++h) {
-        // keys [64h, 64h + 64) -> 32 columns of bf16 pairs at column 32h
-        uint32_t pk[32];
-#pragma unroll
-        for (int qq = 0; qq < 2; ++qq) {
-          const int q = 2 * h + qq;
-          ps2[q] = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const float2 x = ffma2(make_float2(__uint_as_float(sr[q][c]), __uint_as_float(sr[q][c + 1])),
-                                   sl2v, nm2);
-            float2 pv;
-            pv.x = ex2_approx(x.x);
-            pv.y = ex2_approx(x.y);
-            ps2[q] = fadd2(ps2[q], pv);
-            pk[qq * 16 + (c >> 1)] = pack_bf16x2(pv.x, pv.y);
-          }
-        }
-        tmem_st32(tS + h * 32, pk);
-        if (tr && h == 0) FA_TRACE_MARK(1 + t, it, 3);
-      }
-      // the rescale waits until the scores have left the registers
-      if (rescale_o) rescale_o_rows(tO, alpha);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&p_full[t]);
-      float2 psum;
-      if constexpr (kQ32 == 4)
-        psum = fadd2(fadd2(ps2[0], ps2[1]), fadd2(ps2[2], ps2[3]));
-      else
-        psum = fadd2(ps2[0], ps2[1]);
-      l_sum = l_sum * alpha + (psum.x + psum.y);
-      if (tr) FA_TRACE_MARK(1 + t, it, 4);
-    }
-
-    // ------------------------------------------------------------ epilogue
-    if (ok && tile_active[t]) ok = mbar_wait(&o_full[t], 0, abort_flag, status, tmo, kSiteO);
-    const bool failed = named_bar_or(1 + t, kBM, !ok);
-    if (!failed && SPLIT) {
-      // partial state of this key range: u / l (fp32) and its LSE; a range
-      // with no allowed key for this row gives LSE = -inf and weight 0 in
-      // the merge
-      tc_fence_after();
-      const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
-      const float lse_val = l_sum > 0.f ? (m_ref + log2f(l_sum)) * 0.69314718055994530942f : -INFINITY;
-      const size_t prow = (static_cast<size_t>(split) * p.BH + bh) * p.N + row;
-      float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D);
-      const bool row_ok =
-          row < p.N &&
-          in_bounds(split < p.num_splits && bh < p.BH && prow < static_cast<size_t>(p.num_splits) * p.BH * p.N,
-                    kCheckPartial);
-      if (row_ok) p.lse_part[prow] = lse_val;
-      if (tile_active[t]) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
+  } else if (warp >= kSoftmaxWarp0) {
+    regs_alloc<kRegsSoftmax>();
+    if (QT == 2 || warp >= kSoftmaxWarp0 + 4) {  // (with one query tile, slot 0 is unused)
+      // ------------------------------------------------------------ softmax
+      const int t = (warp - kSoftmaxWarp0) >> 2;  // query tile of this warpgroup
+      const int wq = warp & 3;                    // TMEM lane quarter
+      const int r = wq * 32 + lane;               // row inside the tile
+      const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+      const uint32_t tS = tmem + lane_base + t * BN;
+      const uint32_t tO = tmem + lane_base + C::kColO + t * D;
+      const float sl2 = p.scale_log2;
+      // O_t holds the product through the previous tile (that MMA finished
+      // before S_t of this tile was committed): rescale this thread's row of
+      // it in place, before P of this tile releases the next PV product.
+      auto rescale_o_rows = [&](uint32_t taddr, float a) {
+  #pragma unroll
+        for (int cc = 0; cc < D / 16; ++cc) {
+          uint32_t o[16];
+          tmem_ld16(taddr + cc * 16, o);
           tmem_wait_ld();
-          if (row_ok) {
-#pragma unroll
-            for (int g = 0; g < 8; ++g)
-              dst[c * 8 + g] = make_float4(__uint_as_float(o[4 * g]) * inv_l, __uint_as_float(o[4 * g + 1]) * inv_l,
-                                           __uint_as_float(o[4 * g + 2]) * inv_l, __uint_as_float(o[4 * g + 3]) * inv_l);
-          }
+  #pragma unroll
+          for (int kx = 0; kx < 16; ++kx) o[kx] = __float_as_uint(__uint_as_float(o[kx]) * a);
+          tmem_st16(taddr + cc * 16, o);
         }
-      } else if (row_ok) {
-#pragma unroll
-        for (int g = 0; g < D / 4; ++g) dst[g] = make_float4(0.f, 0.f, 0.f, 0.f);
+      };
+
+      bool ok = true;
+      if (p.debug & 1u) {
+        ok = __all_sync(0xffffffffu, mbar_wait(never, 0, abort_flag, status, tmo, kSiteDebug));
       }
-    } else if (!failed) {
-      tc_fence_after();
-      const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
-      if (p.lse != nullptr && row < p.N && in_bounds(bh < p.BH && row >= 0, kCheckLse)) {
+      int s_seen = 0;   // S_t products consumed, over all items
+      int o_seen = 0;   // O_t completions consumed, over all items
+      int trace_it = 0;
+      int w = static_cast<int>(blockIdx.x);
+      for (int k = 0;; ++k) {
+        const Unit u = unit_of<CAUSAL, SPLIT, SPARSE, BN, QT>(p, w);
+        const int row0 = u.q0 + t * kBM;
+        const int row = row0 + r;  // query index in the head
+        const int bh = u.bh;
+        const int n_iter = u.n_iter;
+        const int first = t ? u.first_it[1] : u.first_it[0];
+        const bool active = t ? u.active[1] : u.active[0];
+        const int kv_top = SPARSE ? 0 : u.kv_end - 1;
+        const int* const blk = u.blk;
+        // last key this row may see
+        const int key_limit = CAUSAL ? min(row, p.N - 1) : p.N - 1;
+        auto kv_tile = [&](int it) { return SPARSE ? __ldg(blk + n_iter - 1 - it) : kv_top - it; };
+        float m_ref = -INFINITY;  // reference maximum, log2 units of scaled scores
+        float l_sum = 0.f;        // running denominator relative to m_ref
+        for (int it = first; it < n_iter && ok; ++it) {
+          const int li = it - first;
+          int j = kv_tile(it);
+          // a block-sparse entry out of range or out of order contributes nothing
+          bool bad = false;
+          if (SPARSE) {
+            bad = j < 0 || j >= p.n_kv || (it > 0 && j >= kv_tile(it - 1));
+            if (bad) {
+              if ((threadIdx.x & 127) == 0) atomicOr(&g_device_status, kStatusLayout);
+              j = 0;
+            }
+          }
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(&s_full[t], static_cast<uint32_t>(s_seen) & 1u, abort_flag, status, tmo, kSiteS));
+          if (!ok) break;
+          ++s_seen;
+          const bool tr = lane == 0 && (warp & 3) == 0;
+          if (tr) FA_TRACE_MARK(1 + t, trace_it + it, 0);
+          tc_fence_after();
+          constexpr int kQ32 = BN / 32;  // 32-key groups of a tile
+          uint32_t sr[kQ32][32];
+  #pragma unroll
+          for (int q = 0; q < kQ32; ++q) tmem_ld32(tS + q * 32, sr[q]);
+          tmem_wait_ld();
+          if (tr) FA_TRACE_MARK(1 + t, trace_it + it, 1);
+
+          const int kbase = j * BN;
+          const bool masked = bad || (kbase + BN > p.N) || (CAUSAL && kbase + BN - 1 > row0);
+          if (masked) {
+            const int lim = bad ? -1 : key_limit;
+  #pragma unroll
+            for (int q = 0; q < kQ32; ++q)
+  #pragma unroll
+              for (int cc = 0; cc < 32; ++cc)
+                if (kbase + q * 32 + cc > lim) sr[q][cc] = __float_as_uint(-INFINITY);
+          }
+          // row maximum of the raw scores (scale > 0 keeps the argmax): BN/16
+          // independent chains of three-input maxima
+          constexpr int kChains = BN / 16;
+          float mx[kChains];
+  #pragma unroll
+          for (int kx = 0; kx < kChains; ++kx) mx[kx] = __uint_as_float(sr[kx >> 1][(kx & 1) * 16]);
+  #pragma unroll
+          for (int kx = 0; kx < kChains; ++kx) {
+            const uint32_t* v = &sr[kx >> 1][(kx & 1) * 16];
+  #pragma unroll
+            for (int cc = 1; cc < 15; cc += 2)
+              mx[kx] = fmax3(mx[kx], __uint_as_float(v[cc]), __uint_as_float(v[cc + 1]));
+            mx[kx] = fmaxf(mx[kx], __uint_as_float(v[15]));
+          }
+          float m_all;
+          if constexpr (kChains == 8)
+            m_all = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+          else
+            m_all = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]);
+          const float m_tile = m_all * sl2;
+          if (tr) FA_TRACE_MARK(1 + t, trace_it + it, 2);
+          // raise the reference maximum only when this tile exceeds it by > 2^8
+          const bool raise = m_tile > m_ref + kRescaleThreshold;
+          float alpha = 1.f;
+          if (raise) {
+            alpha = ex2_approx(m_ref - m_tile);  // 0 while m_ref is -inf
+            m_ref = m_tile;
+          }
+          const bool rescale_o = li > 0 && __any_sync(0xffffffffu, raise);
+          const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+          const float2 sl2v = make_float2(sl2, sl2);
+          const float2 nm2 = make_float2(neg_m, neg_m);
+          float2 ps2[kQ32];
+          // p = 2^(s * scale * log2 e - m), written as bf16 pairs over the first
+          // BN/2 columns of S_t, 64 keys at a time, and published whole on
+          // p_full[t].
+  #pragma unroll
+          for (int h = 0; h < BN / 64; ++h) {
+            // keys [64h, 64h + 64) -> 32 columns of bf16 pairs at column 32h
+            uint32_t pk[32];
+  #pragma unroll
+            for (int qq = 0; qq < 2; ++qq) {
+              const int q = 2 * h + qq;
+              ps2[q] = make_float2(0.f, 0.f);
+  #pragma unroll
+              for (int cc = 0; cc < 32; cc += 2) {
+                const float2 x = ffma2(make_float2(__uint_as_float(sr[q][cc]), __uint_as_float(sr[q][cc + 1])),
+                                       sl2v, nm2);
+                float2 pv;
+                pv.x = ex2_approx(x.x);
+                pv.y = ex2_approx(x.y);
+                ps2[q] = fadd2(ps2[q], pv);
+                pk[qq * 16 + (cc >> 1)] = pack_bf16x2(pv.x, pv.y);
+              }
+            }
+            tmem_st32(tS + h * 32, pk);
+            if (tr && h == 0) FA_TRACE_MARK(1 + t, trace_it + it, 3);
+          }
+          // the rescale waits until the scores have left the registers
+          if (rescale_o) rescale_o_rows(tO, alpha);
+          // every lane's stores have completed; one arrival per warp
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_full[t]);
+          if (lane == 0 && wq != 0) FA_TRACE_MARK(1 + t, trace_it + it, 4 + wq);
+          float2 psum;
+          if constexpr (kQ32 == 4)
+            psum = fadd2(fadd2(ps2[0], ps2[1]), fadd2(ps2[2], ps2[3]));
+          else
+            psum = fadd2(ps2[0], ps2[1]);
+          l_sum = l_sum * alpha + (psum.x + psum.y);
+          if (tr) FA_TRACE_MARK(1 + t, trace_it + it, 4);
+        }
+        trace_it += n_iter;
+
+        // ---------------------------------------------------------- epilogue
+        if (ok && active) {
+          ok = mbar_wait(&o_full[t], static_cast<uint32_t>(o_seen) & 1u, abort_flag, status, tmo, kSiteO);
+          ++o_seen;
+        }
+        if (named_bar_or(1 + t, kBM, !ok)) break;
+        tc_fence_after();
+        const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
         const float lse2 = l_sum > 0.f ? m_ref + log2f(l_sum) : -INFINITY;
-        p.lse[static_cast<size_t>(bh) * p.N + row] = lse2 * 0.69314718055994530942f;
-      }
-      // O_t / l -> bf16 -> the Q_t buffer (no MMA reads it any more), laid
-      // out as the 128-byte-swizzled boxes the store tensor map expects.
-      uint8_t* stage = sQ + t * QB;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        if (tile_active[t]) {
-          tmem_ld32(tO + c * 32, o);
-          tmem_wait_ld();
-        } else {  // no retained key (block-sparse): O = 0
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = 0u;
+        if (SPLIT) {
+          // partial state of this key range: u / l (fp32) and its LSE; a range
+          // with no allowed key for this row gives LSE = -inf and weight 0 in
+          // the merge
+          const size_t prow = (static_cast<size_t>(u.split) * p.BH + bh) * p.N + row;
+          float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D);
+          const bool row_ok =
+              row < p.N &&
+              in_bounds(u.split < p.num_splits && bh < p.BH && prow < static_cast<size_t>(p.num_splits) * p.BH * p.N,
+                        kCheckPartial);
+          if (row_ok) p.lse_part[prow] = lse2 * 0.69314718055994530942f;
+  #pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            if (active) {
+              tmem_ld32(tO + cc * 32, o);
+              tmem_wait_ld();
+            } else {
+  #pragma unroll
+              for (int kx = 0; kx < 32; ++kx) o[kx] = 0u;
+            }
+            if (row_ok) {
+  #pragma unroll
+              for (int g = 0; g < 8; ++g)
+                dst[cc * 8 + g] = make_float4(__uint_as_float(o[4 * g]) * inv_l, __uint_as_float(o[4 * g + 1]) * inv_l,
+                                              __uint_as_float(o[4 * g + 2]) * inv_l, __uint_as_float(o[4 * g + 3]) * inv_l);
+            }
+          }
+        } else {
+          if (p.lse != nullptr && row < p.N && in_bounds(bh < p.BH && row >= 0, kCheckLse))
+            p.lse[static_cast<size_t>(bh) * p.N + row] = lse2 * 0.69314718055994530942f;
+          // O_t / l -> bf16, 64 columns at a time through this warp's staging
+          // box (its 32 rows, laid out as the 128-byte swizzle of the store
+          // tensor map), written out by a TMA store; rows past N are clipped
+          // by the store.  The Q buffers stay free for the next item's loads.
+          uint8_t* stage = sO + (warp - kSoftmaxWarp0) * C::kOStageBytes;
+          const int wrow0 = row0 + wq * 32;
+          uint8_t* rowp = stage + lane * 128;
+  #pragma unroll
+          for (int ch = 0; ch < D / 64; ++ch) {
+  #pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              uint32_t o[32];
+              if (active) {
+                tmem_ld32(tO + ch * 64 + h * 32, o);
+                tmem_wait_ld();
+              } else {  // no retained key (block-sparse): O = 0
+  #pragma unroll
+                for (int kx = 0; kx < 32; ++kx) o[kx] = 0u;
+              }
+              if (h == 0) {
+                // the previous store from this box has been read out
+                if (lane == 0) bulk_wait_group_read0();
+                __syncwarp();
+              }
+  #pragma unroll
+              for (int gg = 0; gg < 4; ++gg) {
+                const uint32_t* src = &o[gg * 8];
+                uint4 v;
+                v.x = pack_bf16x2(__uint_as_float(src[0]) * inv_l, __uint_as_float(src[1]) * inv_l);
+                v.y = pack_bf16x2(__uint_as_float(src[2]) * inv_l, __uint_as_float(src[3]) * inv_l);
+                v.z = pack_bf16x2(__uint_as_float(src[4]) * inv_l, __uint_as_float(src[5]) * inv_l);
+                v.w = pack_bf16x2(__uint_as_float(src[6]) * inv_l, __uint_as_float(src[7]) * inv_l);
+                const int gran = (h * 4 + gg) ^ (lane & 7);
+                if (in_bounds(rowp + gran * 16 >= stage && rowp + gran * 16 + 16 <= stage + C::kOStageBytes,
+                              kCheckStage))
+                  *reinterpret_cast<uint4*>(rowp + gran * 16) = v;
+              }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && wrow0 < p.N && in_bounds(wrow0 >= 0 && bh < p.BH, kCheckStore)) {
+              tma_store_3d(&tmO, stage, ch * 64, wrow0, bh);
+              bulk_commit_group();
+            }
+          }
         }
-        uint8_t* rowp = stage + (c >> 1) * kChunkBytes + r * 128;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(o[8 * g + 0]) * inv_l, __uint_as_float(o[8 * g + 1]) * inv_l);
-          v.y = pack_bf16x2(__uint_as_float(o[8 * g + 2]) * inv_l, __uint_as_float(o[8 * g + 3]) * inv_l);
-          v.z = pack_bf16x2(__uint_as_float(o[8 * g + 4]) * inv_l, __uint_as_float(o[8 * g + 5]) * inv_l);
-          v.w = pack_bf16x2(__uint_as_float(o[8 * g + 6]) * inv_l, __uint_as_float(o[8 * g + 7]) * inv_l);
-          const int gran = ((c & 1) * 4 + g) ^ (r & 7);
-          if (in_bounds(rowp + gran * 16 >= stage && rowp + gran * 16 + 16 <= stage + QB, kCheckStage))
-            *reinterpret_cast<uint4*>(rowp + gran * 16) = v;
-        }
+        // the next item; the warps of this warpgroup agree on going on
+        // before any of them reaches the next item's barriers
+        const bool got =
+            __all_sync(0xffffffffu, mbar_wait(&sched_full[k & 1], static_cast<uint32_t>(k >> 1) & 1u, abort_flag,
+                                              status, tmo, kSiteSched));
+        const int next = got ? sched_item[k & 1] : -1;
+        __syncwarp();
+        if (got && lane == 0) mbar_arrive(&sched_empty[k & 1]);
+        if (named_bar_or(1 + t, kBM, !got) || next < 0) break;
+        w = next;
       }
-      fence_proxy_async_smem();
-      named_bar_sync(1 + t, kBM);
-      if (r == 0 && row0 < p.N) {
-        for (int c = 0; c < C::kChunks; ++c)
-          if (in_bounds(row0 >= 0 && bh < p.BH, kCheckStore))
-            tma_store_3d(&tmO, stage + c * kChunkBytes, c * 64, row0, bh);
-        bulk_commit_group();
-        bulk_wait_group_read0();
-      }
+      // the staging box has been read out before the CTA's shared memory goes
+      if (!SPLIT && lane == 0) bulk_wait_group_read0();
     }
   }
 
@@ -762,15 +956,18 @@ fa_status launch(const void* Q, const void* K, const void* V, void* O, FwdParams
   prm.n_kv = (N + BN - 1) / BN;
   CUtensorMap mq, mk, mv, mo;
   if (!make_map_cached(&mq, Q, D, N, BH, kBM) || !make_map_cached(&mk, K, D, N, BH, BN) ||
-      !make_map_cached(&mv, V, D, N, BH, BN) || !make_map_cached(&mo, O, D, N, BH, kBM)) {
+      !make_map_cached(&mv, V, D, N, BH, BN) || (!SPLIT && !make_map_cached(&mo, O, D, N, BH, 32))) {
     snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed");
     return FA_ERR_CUDA;
   }
   const long long rows_per_block = static_cast<long long>(QT) * kBM;
   prm.n_qblk = static_cast<int>((N + rows_per_block - 1) / rows_per_block);
   const long long units = static_cast<long long>(BH) * prm.n_qblk;
-  const long long grid = units * (SPLIT ? prm.num_splits : 1);
-  if (grid > 0x7fffffffll) return FA_ERR_SHAPE;
+  const long long items = units * (SPLIT ? prm.num_splits : 1);
+  if (items > 0x7fffffffll) return FA_ERR_SHAPE;
+  // one CTA per item; each running CTA takes over the items of CTAs not yet
+  // launched, so in practice one CTA per SM runs them all
+  const long long grid = items;
   constexpr int slot = (QT == 1 ? 64 : 0) + (BN == 64 ? 32 : 0) + (SPARSE ? 16 : 0) + (D == 128 ? 8 : 0) +
                        (CAUSAL ? 4 : 0) + (SPLIT ? 1 : 0);
   auto kern = fa_fwd_kernel<D, CAUSAL, SPLIT, SPARSE, BN, QT>;
@@ -785,6 +982,7 @@ fa_status launch(const void* Q, const void* K, const void* V, void* O, FwdParams
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
+  if (SPLIT) mo = mq;  // (unused: the partial states are plain stores)
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, prm);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");

@@ -165,6 +165,56 @@ __device__ __forceinline__ void bulk_wait_group_read0() {
 }
 
 // ---------------------------------------------------------------------------
+// register reallocation between warpgroups
+// ---------------------------------------------------------------------------
+// Every warp of a warpgroup executes the same one, converged.  The registers
+// a warpgroup gives up go to a pool that those asking for more draw from, so
+// the new counts of all warpgroups must add up to no more than the block was
+// launched with.
+template <uint32_t kRegs>
+__device__ __forceinline__ void regs_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <uint32_t kRegs>
+__device__ __forceinline__ void regs_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+
+// ---------------------------------------------------------------------------
+// cluster launch control: take over the work of a CTA not yet launched
+// ---------------------------------------------------------------------------
+// Asks the hardware to cancel the launch of the next pending CTA of this
+// grid (each CTA is a cluster of one here).  The 16-byte answer is written to
+// `resp` (16-byte aligned shared memory) and completes 16 transaction bytes
+// on `bar`, whose arrival the caller has registered with expect_tx.  After an
+// answer that says "not cancelled" no further request may be made.
+__device__ __forceinline__ void clc_try_cancel(void* resp, uint64_t* bar) {
+  asm volatile(
+      "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];" ::"r"(
+          smem_addr(resp)),
+      "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Reads an answer of clc_try_cancel: true and the x index of the cancelled
+// CTA when a launch was cancelled (its work is now the caller's), false when
+// no CTA was left to cancel.
+__device__ __forceinline__ bool clc_query(const void* resp, uint32_t* ctaid_x) {
+  uint32_t ok, x;
+  asm volatile(
+      "{\n\t.reg .b128 r;\n\t.reg .pred p;\n\t"
+      "ld.shared.b128 r, [%2];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t"
+      "clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, r;\n\t}"
+      : "=r"(ok), "=r"(x)
+      : "r"(smem_addr(resp))
+      : "memory");
+  *ctaid_x = x;
+  return ok != 0;
+}
+
+// ---------------------------------------------------------------------------
 // tensor memory
 // ---------------------------------------------------------------------------
 // Warp-wide: allocate `ncols` TMEM columns (power of two >= 32); the base

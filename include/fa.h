@@ -76,7 +76,7 @@ fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
 
 /*
  * fa_fwd_splitkv -- the same result as fa_fwd, with the key range of every
- * query block divided into num_splits ranges processed by separate CTAs, for
+ * query block divided into num_splits ranges processed as separate work items, for
  * problems with too few query blocks to fill the GPU.  Each range leaves a
  * partial state -- its normalised output u/l and its log-sum-exp -- and a
  * second kernel merges the states of a row: with M = max_s LSE_s and
@@ -191,7 +191,7 @@ fa_status fa_fwd_splitkv_noalloc(const void* Q, const void* K, const void* V, vo
  * wall-clock time depends on the tile size (interactiveml.org
  * "FlashAttention saves the matrix, not the quadratic work", the suggested
  * experiments: vary tile size and head width).
- *   query_rows  query rows per CTA: 256 (two 128-row tiles whose softmax and
+ *   query_rows  query rows per work item: 256 (two 128-row tiles whose softmax and
  *               MMAs ping-pong, as fa_fwd) or 128 (one tile, no ping-pong);
  *               0 = 256.
  *   key_tile    keys per score tile: 128 (as fa_fwd) or 64; 0 = 128.
