@@ -39,6 +39,7 @@ if ROOT not in sys.path:
 METRIC = "attention fwd TFLOP/s (bf16, 1×B200) and % of dense-BF16 tensor peak"
 DEFAULT_WORKLOAD = "b2h16n8192d128_causal"
 FALLBACK_PEAK_TFLOPS = 1590.0
+FALLBACK_PEAK_SUSTAINED_TFLOPS = 1400.0
 L2_BYTES = 126 * 1024 * 1024
 KERNEL_SOURCES = ["exact_softmax_attention_02_b200/csrc/fa_fwd.cu",
                   "exact_softmax_attention_02_b200/csrc/sm100.cuh"]
@@ -176,6 +177,19 @@ def tensor_peak():
         return float(peaks["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
     except Exception:
         return FALLBACK_PEAK_TFLOPS, "fallback (1.59 PFLOP/s, earlier measurement on this pool)"
+
+
+def tensor_peak_sustained():
+    """The bf16 peak for a kernel timed inside a seconds-long loop under the
+    power cap (MEASURED_PEAKS.json bf16_tflops_sustained), else the pool's
+    earlier figure (about 1.4 PFLOP/s at about 1.3 GHz)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            peaks = json.load(f)
+        return float(peaks["bf16_tflops_sustained"]), "measured (MEASURED_PEAKS.json bf16_tflops_sustained)"
+    except Exception:
+        return FALLBACK_PEAK_SUSTAINED_TFLOPS, "fallback (1.4 PFLOP/s sustained, earlier measurement on this pool)"
 
 
 def hbm_peak():
@@ -375,8 +389,13 @@ def measure_config(name: str, path: str, dev, steps: int = 20, warmup: int = 5):
     ms = sorted(a.elapsed_time(b) for a, b in ev)
     mean_s = sum(ms) / len(ms) / 1e3
     peak, _ = tensor_peak()
+    peak_s, _ = tensor_peak_sustained()
     tf = flops / mean_s / 1e12
-    out = {"path": path, "tflops": tf, "frac": tf / peak, "ms_per_step": 1e3 * mean_s,
+    # frac: against the burst peak; frac_sustained: against the peak a
+    # seconds-long loop holds under the power cap, the fair one for the long
+    # configurations (their timed loop lasts about a second)
+    out = {"path": path, "tflops": tf, "frac": tf / peak, "frac_sustained": tf / peak_s,
+           "ms_per_step": 1e3 * mean_s,
            "ms_min": ms[0], "ms_median": ms[len(ms) // 2], "steps": steps, "warmup": warmup,
            "flops_per_step": flops, "clocks": sampler.summary(),
            "kernel": ("bwd_rowdot + bwd_dkdv_kernel + bwd_dq_kernel" if path == "backward"

@@ -64,6 +64,9 @@ WORKLOADS = {
         Workload("b1h1n32768d128_causal", 1, 1, 32768, 128, True, 6, sample_rows=1024),
         # small enough for multi-pass ncu captures of the materialising comparator
         Workload("b1h4n4096d128_causal", 1, 4, 4096, 128, True, 7, sample_rows=1024),
+        # four of the eight heads of the N = 131072 causal problem: the same
+        # long-context work list at half the size, for multi-pass ncu captures
+        Workload("b1h4n131072d128_causal", 1, 4, 131072, 128, True, 8, sample_rows=1024),
     )
 }
 
