@@ -16,9 +16,13 @@ stamped).  Roles and events, per iteration ``it``:
 - role 0, the MMA issuer: ``3t`` P of query tile t seen, ``3t + 1`` the PV
   products of tile t issued, ``3t + 2`` the next S product of tile t issued and
   committed (t = 0, 1);
-- roles 1 and 2, one thread of the softmax warpgroup of tile 0 and of tile 1:
-  0 S seen in TMEM, 1 S loaded into registers, 2 row maximum taken, 3 first
-  half of P stored, 4 the tile done (P published, denominator updated).
+- roles 1 and 2, the softmax warpgroup of tile 0 and of tile 1: lane 0 of the
+  warp on TMEM lane quarter 0 stamps 0 S seen in TMEM, 1 S loaded into
+  registers, 2 row maximum taken, 3 first half of P stored, 4 the tile done
+  (P published, denominator updated); lane 0 of the warps on quarters 1, 2, 3
+  stamps 5, 6, 7 when its warp has published P;
+- role 3, the MMA issuer again: 0 the V tile of the iteration landed, 1 the
+  next K tile landed.
 
 The summary averages over iterations whose stamps are all present, leaving out
 the first and last few, where the pipeline fills and drains.
@@ -79,7 +83,23 @@ def summarize(trace: np.ndarray, cta: int = 0, skip_head: int = 4, skip_tail: in
             "to_next_p0": mean(lambda i: mma[i + 1, 0] - mma[i, 5]),
         },
         "s0_issued_to_softmax_sees_it": mean(lambda i: sm0[i + 1, 0] - mma[i, 2]),
+        **publish_lag(t, its),
     }
+
+
+def publish_lag(t: np.ndarray, its) -> dict:
+    """How long after the first warp of a softmax warpgroup each of its four
+    warps published P (mean cycles over the iterations where all four stamped),
+    per query tile; empty when the trace has no per-warp stamps."""
+    out = {}
+    for tile in (0, 1):
+        pubs = t[1 + tile, :, 4:8]
+        rows = [i for i in its if (pubs[i] > 0).all()]
+        if rows:
+            p = pubs[rows].astype(np.float64)
+            lag = (p - p.min(axis=1, keepdims=True)).mean(axis=0)
+            out[f"publish_lag_tile{tile}"] = [float(x) for x in lag]
+    return out
 
 
 def record(workload: str, out: str | None) -> np.ndarray:

@@ -34,6 +34,17 @@ def test_summary_phase_lengths():
     assert s["iterations"] == 20 - 4 - 3
 
 
+def test_publish_lag_per_warp():
+    tr = _synthetic()
+    for it in range(20):
+        base = 10_000 + it * 1000
+        # warps on quarters 1, 2, 3 publish 20, 0 and 40 cycles after quarter 0 (at +100)
+        tr[0, 1, it, 5:8] = base + 100 + np.array([20, 0, 40])
+    s = pt.summarize(tr, cta=0)
+    assert s["publish_lag_tile0"] == pytest.approx([0, 20, 0, 40])
+    assert "publish_lag_tile1" not in s
+
+
 def test_missing_stamps_are_left_out():
     tr = _synthetic()
     tr[0, 1, 8, 3] = 0  # one lost stamp: iteration 8 no longer counts
