@@ -11,23 +11,24 @@
 //
 // Three kernels:
 //   bwd_rowdot   D = rowsum(dO * O) and LSE * log2(e), one warp per row,
-//                into a workspace padded to whole 128-row tiles (HBM-bound).
-//   bwd_dkdv     one CTA per 128-key tile: S^T = K Q^T and dP^T = V dO^T into
-//                TMEM, P^T and dS^T formed in place (bf16), then
-//                dV += P^T dO and dK += dS^T Q accumulate in TMEM over the
-//                query tiles (tcgen05, A operands from TMEM).
-//   bwd_dq       one CTA per 128-query tile: S = Q K^T and dP = dO V^T, dS in
-//                place, dQ += dS K over the key tiles.
-// CTA layout of the two tiled kernels (384 threads): warp 0 TMA producer,
-// warp 1 TMEM owner and MMA issuer, warps 4-11 elementwise step and epilogue
-// (two threads per TMEM lane, i.e. per row).  The elementwise threads work
-// through each tile a quarter (32 columns) at a time and release every
-// quarter to the MMA issuer on its own barrier, so that the accumulating
-// products of one quarter overlap the elementwise step of the next.  The
-// MMAs are all N = 128 (S, dP) or N = d (accumulators): issuing a
-// tcgen05.mma takes its thread about as long as an M = 128, N = 128, K = 16
-// product runs, so narrower products would leave the tensor core waiting on
-// issue.
+//                into a workspace padded to whole 128-row tiles, and the fp32
+//                dQ accumulator set to zero (HBM-bound).
+//   bwd_dkdv     one CTA per 128-key tile, over the query tiles that see it:
+//                S^T = K Q^T and dP^T = V dO^T into TMEM, P^T and dS^T formed
+//                in place (bf16); dV += P^T dO and dK += dS^T Q accumulate in
+//                TMEM; dQ_i = dS K, the tile's share of the query tile's dQ,
+//                is formed in TMEM and added into the fp32 accumulator in
+//                global memory (reductions at L2).  Every product of the
+//                gradient is computed once.
+//   bwd_dq_convert  dQ = scale * accumulator, to bf16.
+// CTA layout of bwd_dkdv (384 threads): warp 0 TMA producer, warp 1 TMEM
+// owner and MMA issuer, warps 4-11 elementwise step, dQ reductions and
+// epilogue (two threads per TMEM lane, i.e. per row).  The elementwise
+// threads work through each tile a quarter (32 columns) at a time
+// and release every quarter to the MMA issuer on its own barrier, so that the
+// accumulating products of one quarter overlap the elementwise step of the
+// next.  The MMAs are N = 128 (S, dP) or N = d (accumulators): an M = 128
+// tcgen05.mma costs about the same at N = 64 as at N = 128.
 // Every wait is bounded as in the forward kernel.
 
 #include <cuda.h>
@@ -54,11 +55,12 @@ constexpr int kElemThreads = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kChunkBytes = kTile * 64 * 2;  // one 64-wide, 128-row swizzled box: 16 KB
 
-enum : uint32_t { kSiteLoad = 0, kSiteStage = 1, kSiteS = 2, kSiteDs = 3, kSiteO = 4 };
+enum : uint32_t { kSiteLoad = 0, kSiteStage = 1, kSiteS = 2, kSiteDs = 3, kSiteO = 4, kSiteDq = 5 };
 
 struct BwdParams {
   const float* lse2;  // [BH][n_pad] the forward's LSE times log2(e); +inf past N
   const float* dd;    // [BH][n_pad] D = rowsum(dO * O); 0 past N
+  float* dq_acc;      // [BH][n_pad][d] fp32: dS K summed over the key tiles by reduce-adds
   int N;
   int n_pad;          // N rounded up to a multiple of 128
   int BH;
@@ -101,6 +103,12 @@ constexpr uint32_t kColS = 0, kColDP = 128, kColAcc = 256;
 // TMEM column of the packed bf16 operand for K-step kk (16 queries or keys):
 // quarter kk / 2, half kk % 2
 __device__ __forceinline__ uint32_t packed_col(int kk) { return (kk >> 1) * 32 + (kk & 1) * 16; }
+
+// *p += v, four fp32 adds performed at L2 (no value returned)
+__device__ __forceinline__ void red_add_v4(float* p, float4 v) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
 
 // Work order shared by the tiled kernels: heads in groups, inside a group the
 // tiles with the most work first, cycling over the group's heads.
@@ -180,9 +188,14 @@ __device__ __forceinline__ void ds_16(const float (&p)[16], const uint32_t (&dp)
 // one is computed, and its dP while the current stores drain; P (optional)
 // and dS go back as bf16 pairs over the first 8 of each thread's 16 columns,
 // and each quarter is released on ready[q] once its stores have completed.
-template <bool WRITE_P, bool MASK, typename Col, typename Allowed, typename Wait>
+// DS_SMEM: dS also goes to shared memory as the A operand of dQ_i = dS K:
+// [keys][queries] (query-contiguous, two 64-query chunks of 128-byte rows in
+// the 128-byte swizzle), row r = the thread's key; ds_row points at row r of
+// the first chunk.
+template <bool WRITE_P, bool MASK, bool DS_SMEM, typename Col, typename Allowed, typename Wait>
 __device__ __forceinline__ bool p_ds_tile(uint32_t tS, uint32_t tDP, int h, float sl2, Col col,
-                                          Allowed allowed, uint64_t* ready, Wait dp_ready) {
+                                          Allowed allowed, uint64_t* ready, Wait dp_ready,
+                                          uint8_t* ds_row = nullptr, int r = 0) {
   uint32_t s[2][16], dp[16];
   tmem_ld16(tS + h * 16, s[0]);
   tmem_wait_ld_reg16(s[0]);
@@ -203,6 +216,14 @@ __device__ __forceinline__ bool p_ds_tile(uint32_t tS, uint32_t tDP, int h, floa
     if (q < 3) tmem_ld16(tDP + c0 + kQuarter, dp);
     if (WRITE_P) tmem_st8(tS + c0, pk);
     tmem_st8(tDP + c0, dk);
+    if (DS_SMEM) {
+      // queries c0..c0+15 = 16-byte granules gb, gb + 1 of the row in chunk q / 2
+      uint8_t* rowp = ds_row + (q >> 1) * kChunkBytes;
+      const int gb = (q & 1) * 4 + h * 2;
+      *reinterpret_cast<uint4*>(rowp + ((gb ^ (r & 7)) * 16)) = make_uint4(dk[0], dk[1], dk[2], dk[3]);
+      *reinterpret_cast<uint4*>(rowp + (((gb + 1) ^ (r & 7)) * 16)) = make_uint4(dk[4], dk[5], dk[6], dk[7]);
+      fence_proxy_async_smem();  // visible to the tensor core's reads
+    }
     tmem_wait_st();
     tc_fence_before();
     mbar_arrive(&ready[q]);
@@ -244,11 +265,20 @@ template <int D>
 __global__ void __launch_bounds__(256)
     bwd_rowdot_kernel(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __restrict__ dO,
                       const float* __restrict__ lse, float* __restrict__ lse2, float* __restrict__ dd,
-                      int N, int n_pad, long long rows_pad) {
+                      float* __restrict__ dq_acc, int N, int n_pad, long long rows_pad) {
   constexpr int kPer = D / 32;
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows_pad) return;
+  // the dQ accumulator row starts at zero (padding rows too: they receive
+  // reduce-adds of zeros)
+  {
+    float* z = dq_acc + row * D + lane * kPer;
+    if constexpr (kPer == 4)
+      *reinterpret_cast<float4*>(z) = make_float4(0.f, 0.f, 0.f, 0.f);
+    else
+      *reinterpret_cast<float2*>(z) = make_float2(0.f, 0.f);
+  }
   const long long bh = row / n_pad;
   const int q = static_cast<int>(row - bh * n_pad);
   if (q >= N) {  // padding: P = 0 there
@@ -285,18 +315,38 @@ struct DkdvCfg {
   static constexpr int kTileBytes = kTile * D * 2;
   static constexpr int kStages = D == 128 ? 2 : 4;  // each stage: Q_i and dO_i (+ LSE2_i, D_i)
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kSmemTiles = 2 * kTileBytes + kStages * kStageBytes;  // K, V, ring
+  // dS of the current tile (bf16, [keys][queries] in two 64-query chunks):
+  // the A operand of dQ_i = dS K; once that product has finished, the
+  // elementwise warps transpose dQ_i's rows through it, one 32-row x
+  // 32-column (fp32) box per warp at a time
+  static constexpr int kDsBytes = 2 * kChunkBytes;
+  static constexpr int kBoxBytes = 32 * 128;
+  static_assert((kElemThreads / 32) * kBoxBytes <= kDsBytes, "the transposition boxes fit the dS buffer");
+  static constexpr int kSmemTiles = 2 * kTileBytes + kStages * kStageBytes + kDsBytes;  // K, V, ring, dS
   static constexpr int kLdBytes = kStages * 2 * kTile * 4;
-  static constexpr int kNumBars = 1 + 2 * kStages + 2 + 4 + 1 + 1;
-  static constexpr int kSmemBytes = kSmemTiles + kLdBytes + kNumBars * 8 + 16 + 1024;
+  static constexpr int kNumBars = 1 + 2 * kStages + 2 + 4 + 1 + 1 + 2;
+  // No alignment slack: at d = 128 it would not fit in 227 KB.  The kernel
+  // checks that its dynamic shared memory starts 1024-aligned instead.
+  static constexpr int kSmemBytes = kSmemTiles + kLdBytes + kNumBars * 8 + 16;
+  // the dQ_i product in TMEM: over S^T at d = 128 (all 512 columns are
+  // otherwise in use), in the 128 columns past the accumulators at d = 64
+  static constexpr uint32_t kColDQ = D == 128 ? kColS : kColAcc + 2 * D;
+  static_assert(kColDQ + D <= kTmemCols, "dQ_i fits in TMEM");
 };
 
-// Per query tile i: S^T = K Q_i^T and dP^T = V dO_i^T (N = 128) into TMEM;
-// the elementwise threads then form P^T and dS^T a quarter (32 queries) at a
-// time and release each quarter on its own barrier, so that dV += P^T dO and
-// dK += dS^T Q run on one quarter while the next is being formed.  tcgen05
-// MMAs of one thread run in issue order, so the S^T of tile i+1 may be issued
-// right after the products that read tile i's P^T and dS^T.
+// One CTA per 128-key tile j; per query tile i (the ones that see tile j):
+//   S^T = K Q_i^T and dP^T = V dO_i^T (N = 128) into TMEM;
+//   the elementwise threads form P^T and dS^T a quarter (32 queries) at a
+//   time and release each quarter on its own barrier, so that dV += P^T dO_i
+//   and dK += dS^T Q_i run on one quarter while the next is being formed;
+//   they also write dS to shared memory, and dQ_i = dS K (the tile's share of
+//   dQ for query tile i) is then formed in TMEM, read out by the elementwise
+//   warps and added into the fp32 dQ accumulator in global memory by TMA
+//   reduce-adds.  So every product of the gradient is computed once: no
+//   second pass recomputes S and dP for dQ.
+// tcgen05 MMAs of one thread run in issue order, so dP^T of tile i+1 may be
+// issued right after the products that read tile i's dS^T, and S^T of tile
+// i+1 right after dQ_i has been read out of the columns they share (d = 128).
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -306,12 +356,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   using C = DkdvCfg<D>;
   constexpr int S = C::kStages;
   constexpr int TB = C::kTileBytes;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // the swizzled tiles need 1024-byte alignment and there is no slack to
+  // align by hand: refuse to run otherwise (uniformly, before any barrier)
+  if ((smem_addr(smem_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicOr(&g_bwd_status, kStatusBounds);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint8_t* sK = smem;
   uint8_t* sV = smem + TB;
   uint8_t* sRing = smem + 2 * TB;  // stage s: Q_i at +0, dO_i at +TB
+  uint8_t* sDs = sRing + S * C::kStageBytes;
   float* sLd = reinterpret_cast<float*>(smem + C::kSmemTiles);  // stage s: LSE2 [128], D [128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemTiles + C::kLdBytes);
   uint64_t* kv_full = bars;           // K, V landed
@@ -319,10 +375,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* st_empty = st_full + S;   // [S] MMA done with a stage
   uint64_t* s_full = st_empty + S;    // S^T in TMEM
   uint64_t* dp_full = s_full + 1;     // dP^T in TMEM
-  uint64_t* ds_ready = dp_full + 1;   // [4] quarter q of P^T and dS^T in TMEM (256 arrivals)
+  uint64_t* ds_ready = dp_full + 1;   // [4] quarter q of P^T and dS^T in TMEM, dS in SMEM (256 arrivals)
   uint64_t* acc_done = ds_ready + 4;  // dK, dV final
   uint64_t* mma_done = acc_done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* dq_full = mma_done + 1;     // dQ_i in TMEM (dS no longer read)
+  uint64_t* dq_drained = dq_full + 1;   // dQ_i read out of TMEM (one arrival per elementwise warp)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dq_drained + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* status = &g_bwd_status;
   const uint64_t tmo = p.timeout_ns;
@@ -344,6 +402,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int q = 0; q < 4; ++q) mbar_init(&ds_ready[q], kElemThreads);
     mbar_init(acc_done, 1);
     mbar_init(mma_done, 1);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_drained, kElemThreads / 32);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -395,7 +455,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(kTile, kTile, false);
       constexpr uint32_t idAcc = idesc_bf16_f32(kTile, D, true);
-      const uint32_t sk = smem_addr(sK), sv = smem_addr(sV), sr = smem_addr(sRing);
+      constexpr uint32_t idDq = idesc_bf16_f32(kTile, D, true, true);
+      const uint32_t sk = smem_addr(sK), sv = smem_addr(sV), sr = smem_addr(sRing), sds = smem_addr(sDs);
       // X^T = A B^T with A, B both [128 rows][d] K-major tiles
       auto issue_abt = [&](uint32_t d_tmem, uint32_t a, uint32_t b) {
 #pragma unroll
@@ -414,18 +475,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                  (accumulate || kk > 0) ? 1u : 0u);
         }
       };
+      // dQ_i = dS K: A = dS [keys][queries] (M = queries contiguous), B = K
+      // [keys][d] (N = d contiguous); 16 keys (rows) = 2 KB per K-step
+      auto issue_dq = [&]() {
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ss(tmem + C::kColDQ, sw128_desc(sds + kk * 2048, kChunkBytes, 1024),
+                 sw128_desc(sk + kk * 2048, kChunkBytes, 1024), idDq, kk > 0 ? 1u : 0u);
+      };
       bool ok = mbar_wait(kv_full, 0, abort_flag, status, tmo, kSiteLoad);
+      if (ok && n_iter > 0 && (ok = mbar_wait(&st_full[0], 0, abort_flag, status, tmo, kSiteLoad))) {
+        tc_fence_after();
+        issue_abt(tmem + kColS, sk, sr);        // S^T = K Q^T
+        mma_commit(s_full);
+        issue_abt(tmem + kColDP, sv, sr + TB);  // dP^T = V dO^T
+        mma_commit(dp_full);
+      }
       for (int it = 0; it < n_iter && ok; ++it) {
         const int s = it % S;
-        if (!(ok = mbar_wait(&st_full[s], static_cast<uint32_t>(it / S) & 1u, abort_flag, status, tmo, kSiteLoad)))
-          break;
-        BWD_TRACE(0, 0, it, 0);
-        tc_fence_after();
         const uint32_t q = sr + s * C::kStageBytes, dO = q + TB;
-        issue_abt(tmem + kColS, sk, q);   // S^T = K Q^T
-        mma_commit(s_full);
-        issue_abt(tmem + kColDP, sv, dO); // dP^T = V dO^T
-        mma_commit(dp_full);
         BWD_TRACE(0, 0, it, 1);
         for (int qq = 0; qq < 4 && ok; ++qq) {
           if (!(ok = mbar_wait(&ds_ready[qq], static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteDs)))
@@ -437,20 +505,47 @@ __global__ void __launch_bounds__(kThreads, 1)
           issue_acc_q(tmem + kColAcc + D, tmem + kColDP, q, qq, it > 0);  // dK += dS^T Q
         }
         if (!ok) break;
+        // at d = 64 dQ_i has columns of its own: the previous one must have been read out
+        if (D == 64 && it > 0 &&
+            !(ok = mbar_wait(dq_drained, static_cast<uint32_t>(it - 1) & 1u, abort_flag, status, tmo, kSiteDq)))
+          break;
+        issue_dq();
+        mma_commit(dq_full);
         mma_commit(&st_empty[s]);
         BWD_TRACE(0, 0, it, 3);
+        if (it + 1 < n_iter) {
+          const int s1 = (it + 1) % S;
+          const uint32_t q1 = sr + s1 * C::kStageBytes;
+          if (!(ok = mbar_wait(&st_full[s1], static_cast<uint32_t>((it + 1) / S) & 1u, abort_flag, status, tmo,
+                               kSiteLoad)))
+            break;
+          BWD_TRACE(0, 0, it + 1, 0);
+          tc_fence_after();
+          issue_abt(tmem + kColDP, sv, q1 + TB);  // dP^T of the next tile: dK has read this dS^T
+          mma_commit(dp_full);
+          // at d = 128 the next S^T goes where dQ_i is: wait until it is read out
+          if (D == 128 &&
+              !(ok = mbar_wait(dq_drained, static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteDq)))
+            break;
+          tc_fence_after();
+          issue_abt(tmem + kColS, sk, q1);
+          mma_commit(s_full);
+        }
       }
       if (ok) mma_commit(acc_done);
       mma_commit(mma_done);
       mbar_wait_drain(mma_done, 0, tmo);
     }
   } else if (warp >= kElemWarp0) {
-    const int h = (warp - kElemWarp0) >> 2;  // which 16 columns of every quarter
+    const int e = warp - kElemWarp0;  // elementwise warp 0..7
+    const int h = e >> 2;              // which 16 columns of every quarter; which half of dQ_i's columns
     const int wq = warp & 3;
-    const int r = wq * 32 + lane;  // key row inside the tile
+    const int r = wq * 32 + lane;  // key row inside the tile; query row of dQ_i
     const int key = j * kTile + r;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_base + kColS, tDP = tmem + lane_base + kColDP;
+    const uint32_t tDQ = tmem + lane_base + C::kColDQ;
+    uint8_t* box = sDs + e * C::kBoxBytes;  // this warp's transposition box
     const float sl2 = p.scale_log2;
     const bool tr = lane == 0 && wq == 0;
     bool ok = true;
@@ -479,16 +574,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         return __all_sync(0xffffffffu, mbar_wait(dp_full, static_cast<uint32_t>(it) & 1u, abort_flag, status,
                                                  tmo, kSiteS));
       };
-      ok = diag ? p_ds_tile<true, true>(tS, tDP, h, sl2, col, allowed, ds_ready, dp_ready)
-                : p_ds_tile<true, false>(tS, tDP, h, sl2, col, allowed, ds_ready, dp_ready);
+      // (the previous tile's transposition is over: every warp passed the
+      // barrier that ends it)
+      uint8_t* ds_row = sDs + r * 128;
+      ok = diag ? p_ds_tile<true, true, true>(tS, tDP, h, sl2, col, allowed, ds_ready, dp_ready, ds_row, r)
+                : p_ds_tile<true, false, true>(tS, tDP, h, sl2, col, allowed, ds_ready, dp_ready, ds_row, r);
       if (tr) BWD_TRACE(0, 1 + h, it, 1);
+      if (!ok) break;
+      // dQ_i: this thread's query row r, columns [h d/2, (h+1) d/2), 32 at a time
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(dq_full, static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteDq));
+      if (!ok) break;
+      tc_fence_after();
+      constexpr int kRounds = D / 64;
+      uint32_t o[kRounds][32];
+#pragma unroll
+      for (int rd = 0; rd < kRounds; ++rd) tmem_ld32(tDQ + h * (D / 2) + rd * 32, o[rd]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dq_drained);
+      // Added into the fp32 accumulator 32 columns at a time through this
+      // warp's box (the dQ_i product has finished, so dS is no longer read
+      // and its buffer holds the boxes): each lane writes its row (128 bytes,
+      // 16-byte granules rotated by the row to spread the banks), then the
+      // warp reads the box back four rows per instruction, eight lanes per
+      // row, so that every reduction instruction covers four whole 128-byte
+      // lines of the accumulator.
+      float* acc_base = p.dq_acc + (static_cast<size_t>(bh) * p.n_pad + i * kTile + wq * 32) * D + h * (D / 2);
+#pragma unroll
+      for (int rd = 0; rd < kRounds; ++rd) {
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+          *reinterpret_cast<uint4*>(box + lane * 128 + ((g ^ (lane & 7)) * 16)) =
+              make_uint4(o[rd][4 * g], o[rd][4 * g + 1], o[rd][4 * g + 2], o[rd][4 * g + 3]);
+        __syncwarp();
+#pragma unroll
+        for (int k4 = 0; k4 < 8; ++k4) {
+          const int row = k4 * 4 + (lane >> 3), g = lane & 7;
+          const float4 v = *reinterpret_cast<const float4*>(box + row * 128 + ((g ^ (row & 7)) * 16));
+          red_add_v4(acc_base + static_cast<size_t>(row) * D + rd * 32 + g * 4, v);
+        }
+        __syncwarp();  // the box is read before the next round overwrites it
+      }
+      // the next tile's dS goes into the same buffer: every warp must have
+      // read its boxes back first
+      named_bar_sync(3, kElemThreads);
+      if (tr) BWD_TRACE(0, 1 + h, it, 2);
     }
     if (ok) ok = mbar_wait(acc_done, 0, abort_flag, status, tmo, kSiteO);
     const bool failed = named_bar_or(2, kElemThreads, !ok);
     if (!failed && n_iter > 0) {
       tc_fence_after();
-      // K and V are no longer read by any MMA: they stage dK (warps 4-7)
-      // and dV (warps 8-11)
+      // K and V are no longer read by any MMA (the last dQ_i has finished):
+      // they stage dK (warps 4-7) and dV (warps 8-11)
       if (h == 0)
         store_tile<D>(tmem + lane_base + kColAcc + D, p.scale, sK, r, 0, D / 32);
       else
@@ -515,249 +654,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// ---------------------------------------------------------------------------
-// dQ: one CTA per 128-query tile
-// ---------------------------------------------------------------------------
+// dQ = scale * (sum over the key tiles of dS K), fp32 -> bf16, rows < N; one
+// warp per row.
 template <int D>
-struct DqCfg {
-  static constexpr int kChunks = D / 64;
-  static constexpr int kTileBytes = kTile * D * 2;
-  static constexpr int kStages = D == 128 ? 2 : 4;  // each stage: K_j and V_j
-  static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kSmemTiles = 2 * kTileBytes + kStages * kStageBytes;  // Q, dO, ring
-  static constexpr int kNumBars = 1 + 2 * kStages + 2 + 4 + 1 + 1 + 1;
-  static constexpr int kSmemBytes = kSmemTiles + kNumBars * 8 + 16 + 1024;
-  // Q and dO stay in TMEM for the whole CTA, as the A operands of S and dP
-  // (bf16 pairs, d/2 columns each), next to the dQ accumulator
-  static constexpr uint32_t kColQ = kColAcc + D;
-  static constexpr uint32_t kColDO = kColQ + D / 2;
-  static_assert(kColDO + D / 2 <= kTmemCols, "S, dP, dQ, Q and dO fit in TMEM");
-};
-
-// Same quarter pipeline over the key tiles j: S = Q K_j^T, dP = dO V_j^T, dS
-// in place a quarter (32 keys) at a time, dQ += dS K_j per quarter.  Q and
-// dO are copied once into TMEM, so that S and dP are TS products whose only
-// shared-memory operand is the streamed K or V tile (half the operand reads
-// of an SS product).
-template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(kThreads, 1)
-    bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                  const __grid_constant__ CUtensorMap tmdQ, const BwdParams p) {
-  using C = DqCfg<D>;
-  constexpr int S = C::kStages;
-  constexpr int TB = C::kTileBytes;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sdO = smem + TB;
-  uint8_t* sRing = smem + 2 * TB;  // stage s: K at +0, V at +TB
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemTiles);
-  uint64_t* q_full = bars;
-  uint64_t* st_full = bars + 1;
-  uint64_t* st_empty = st_full + S;
-  uint64_t* s_full = st_empty + S;   // S in TMEM
-  uint64_t* dp_full = s_full + 1;    // dP in TMEM
-  uint64_t* ds_ready = dp_full + 1;  // [4]
-  uint64_t* acc_done = ds_ready + 4;
-  uint64_t* mma_done = acc_done + 1;
-  uint64_t* qt_ready = mma_done + 1;  // Q and dO copied into TMEM (256 arrivals)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qt_ready + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint32_t* status = &g_bwd_status;
-  const uint64_t tmo = p.timeout_ns;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int bh, i;
-  tile_of(p, /*heavy_high=*/true, &bh, &i);  // causal: high query tiles see the most keys
-  const int n_iter = CAUSAL ? i + 1 : p.n_tiles;
-
-  if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&st_full[s], 1);
-      mbar_init(&st_empty[s], 1);
-    }
-    mbar_init(s_full, 1);
-    mbar_init(dp_full, 1);
-    for (int q = 0; q < 4; ++q) mbar_init(&ds_ready[q], kElemThreads);
-    mbar_init(acc_done, 1);
-    mbar_init(mma_done, 1);
-    mbar_init(qt_ready, kElemThreads);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      bool ok = true;
-      mbar_arrive_expect_tx(q_full, 2 * TB);
-      for (int c = 0; c < C::kChunks; ++c) {
-        tma_load_3d(sQ + c * kChunkBytes, &tmQ, q_full, c * 64, i * kTile, bh);
-        tma_load_3d(sdO + c * kChunkBytes, &tmdO, q_full, c * 64, i * kTile, bh);
-      }
-      int it = 0;
-      for (; it < n_iter && ok; ++it) {
-        const int s = it % S;
-        const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
-        ok = mbar_wait(&st_empty[s], ph ^ 1u, abort_flag, status, tmo, kSiteStage);
-        if (!ok) break;
-        uint8_t* st = sRing + s * C::kStageBytes;
-        mbar_arrive_expect_tx(&st_full[s], 2 * TB);
-        for (int c = 0; c < C::kChunks; ++c) {
-          tma_load_3d(st + c * kChunkBytes, &tmK, &st_full[s], c * 64, it * kTile, bh);
-          tma_load_3d(st + TB + c * kChunkBytes, &tmV, &st_full[s], c * 64, it * kTile, bh);
-        }
-      }
-      if (!ok) {
-        for (int s = 0; s < S && s < it; ++s) {
-          const int last = s + ((it - 1 - s) / S) * S;
-          mbar_wait_drain(&st_full[s], static_cast<uint32_t>(last / S) & 1u, tmo);
-        }
-        mbar_wait_drain(q_full, 0, tmo);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(kTile, kTile, false);
-      constexpr uint32_t idAcc = idesc_bf16_f32(kTile, D, true);
-      const uint32_t sr = smem_addr(sRing);
-      // X = A B^T with A (Q or dO, 128 rows) in TMEM, B (K or V, 128 rows) K-major in SMEM
-      auto issue_tbt = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-          mma_ts(d_tmem, a_tmem + kk * 8, sw128_desc(b + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
-        }
-      };
-      bool ok = mbar_wait(qt_ready, 0, abort_flag, status, tmo, kSiteLoad);
-      for (int it = 0; it < n_iter && ok; ++it) {
-        const int s = it % S;
-        if (!(ok = mbar_wait(&st_full[s], static_cast<uint32_t>(it / S) & 1u, abort_flag, status, tmo, kSiteLoad)))
-          break;
-        BWD_TRACE(1, 0, it, 0);
-        tc_fence_after();
-        const uint32_t k = sr + s * C::kStageBytes, v = k + TB;
-        issue_tbt(tmem + kColS, tmem + C::kColQ, k);    // S = Q K^T
-        mma_commit(s_full);
-        issue_tbt(tmem + kColDP, tmem + C::kColDO, v);  // dP = dO V^T
-        mma_commit(dp_full);
-        BWD_TRACE(1, 0, it, 1);
-        for (int qq = 0; qq < 4 && ok; ++qq) {
-          if (!(ok = mbar_wait(&ds_ready[qq], static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteDs)))
-            break;
-          if (qq == 0) BWD_TRACE(1, 0, it, 2);
-          BWD_TRACE(1, 0, it, 4 + qq);
-          tc_fence_after();
-          // dQ += dS K: A = dS in TMEM (over dP), B = K tile as [keys][d] (MN-major)
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int kk = 2 * qq + hh;
-            mma_ts(tmem + kColAcc, tmem + kColDP + packed_col(kk), sw128_desc(k + kk * 2048, kChunkBytes, 1024),
-                   idAcc, (it > 0 || kk > 0) ? 1u : 0u);
-          }
-        }
-        if (!ok) break;
-        mma_commit(&st_empty[s]);
-        BWD_TRACE(1, 0, it, 3);
-      }
-      if (ok) mma_commit(acc_done);
-      mma_commit(mma_done);
-      mbar_wait_drain(mma_done, 0, tmo);
-    }
-  } else if (warp >= kElemWarp0) {
-    const int h = (warp - kElemWarp0) >> 2;  // which 16 columns of every quarter
-    const int wq = warp & 3;
-    const int r = wq * 32 + lane;  // query row inside the tile
-    const int row = i * kTile + r;
-    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_base + kColS, tDP = tmem + lane_base + kColDP;
-    const float sl2 = p.scale_log2;
-    const bool tr = lane == 0 && wq == 0;
-    // this row's LSE2 and D (padding rows: +inf and 0, so P = 0)
-    const size_t prow = static_cast<size_t>(bh) * p.n_pad + row;
-    const float lse2 = p.lse2[prow];
-    const float dsub = p.dd[prow];
-    const float4 l4c = make_float4(lse2, lse2, lse2, lse2);
-    const float4 d4c = make_float4(dsub, dsub, dsub, dsub);
-    auto col = [&](int, float4& l4, float4& d4) {
-      l4 = l4c;
-      d4 = d4c;
-    };
-    // this thread's row of Q (h = 0) or dO (h = 1), from its 128-byte-swizzled
-    // tile into TMEM as bf16 pairs in order: the TS products' A layout
-    bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, status, tmo, kSiteLoad));
-    if (ok) {
-      const uint8_t* src = (h == 0 ? sQ : sdO) + r * 128;
-      const uint32_t dst = tmem + lane_base + (h == 0 ? C::kColQ : C::kColDO);
-#pragma unroll
-      for (int c = 0; c < C::kChunks; ++c) {
-        uint32_t w[32];
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          const uint4 v = *reinterpret_cast<const uint4*>(src + c * kChunkBytes + ((g ^ (r & 7)) * 16));
-          w[4 * g] = v.x;
-          w[4 * g + 1] = v.y;
-          w[4 * g + 2] = v.z;
-          w[4 * g + 3] = v.w;
-        }
-        tmem_st32(dst + c * 32, w);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(qt_ready);
-    }
-    for (int it = 0; it < n_iter && ok; ++it) {
-      ok = __all_sync(0xffffffffu,
-                      mbar_wait(s_full, static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteS));
-      if (!ok) break;
-      if (tr) BWD_TRACE(1, 1 + h, it, 0);
-      tc_fence_after();
-      // keys past N need no mask: their K and V rows are zero, so they add
-      // nothing to dQ; the causal diagonal tile does
-      const int k0 = it * kTile;
-      auto allowed = [&](int c) { return k0 + c <= row; };
-      const bool diag = CAUSAL && it == i;
-      auto dp_ready = [&]() {
-        return __all_sync(0xffffffffu, mbar_wait(dp_full, static_cast<uint32_t>(it) & 1u, abort_flag, status,
-                                                 tmo, kSiteS));
-      };
-      ok = diag ? p_ds_tile<false, true>(tS, tDP, h, sl2, col, allowed, ds_ready, dp_ready)
-                : p_ds_tile<false, false>(tS, tDP, h, sl2, col, allowed, ds_ready, dp_ready);
-      if (tr) BWD_TRACE(1, 1 + h, it, 1);
-    }
-    if (ok) ok = mbar_wait(acc_done, 0, abort_flag, status, tmo, kSiteO);
-    const bool failed = named_bar_or(2, kElemThreads, !ok);
-    if (!failed) {
-      tc_fence_after();
-      // Q is no longer read by any MMA: it stages dQ, each half of the
-      // threads taking half of the columns
-      store_tile<D>(tmem + lane_base + kColAcc, p.scale, sQ, r, h * (D / 64), (h + 1) * (D / 64));
-      fence_proxy_async_smem();
-      named_bar_sync(1, kElemThreads);
-      if (h == 0 && r == 0) {
-        for (int c = 0; c < C::kChunks; ++c) tma_store_3d(&tmdQ, sQ + c * kChunkBytes, c * 64, i * kTile, bh);
-        bulk_commit_group();
-        bulk_wait_group_read0();
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+__global__ void __launch_bounds__(256)
+    bwd_dq_convert_kernel(const float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dQ, float scale,
+                          int N, int n_pad, long long rows) {
+  constexpr int kPer = D / 32;
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const long long bh = row / N;
+  const long long q = row - bh * N;
+  const float* src = dq_acc + (bh * n_pad + q) * D + lane * kPer;
+  __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(dQ + row * D + lane * kPer);
+  if constexpr (kPer == 4) {
+    const float4 v = *reinterpret_cast<const float4*>(src);
+    dst[0] = __floats2bfloat162_rn(v.x * scale, v.y * scale);
+    dst[1] = __floats2bfloat162_rn(v.z * scale, v.w * scale);
+  } else {
+    const float2 v = *reinterpret_cast<const float2*>(src);
+    dst[0] = __floats2bfloat162_rn(v.x * scale, v.y * scale);
   }
 }
 
@@ -788,32 +705,31 @@ fa_status launch_bwd(const void* Q, const void* K, const void* V, const void* O,
                      const float* LSE, void* dQ, void* dK, void* dV, float* lse2, float* dd, BwdParams prm,
                      cudaStream_t st) {
   const int N = prm.N, BH = prm.BH;
-  CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv;
+  CUtensorMap mq, mk, mv, mdo, mdk, mdv;
   if (!host::make_map_cached(&mq, Q, D, N, BH, kTile) || !host::make_map_cached(&mk, K, D, N, BH, kTile) ||
       !host::make_map_cached(&mv, V, D, N, BH, kTile) || !host::make_map_cached(&mdo, dO, D, N, BH, kTile) ||
-      !host::make_map_cached(&mdq, dQ, D, N, BH, kTile) || !host::make_map_cached(&mdk, dK, D, N, BH, kTile) ||
-      !host::make_map_cached(&mdv, dV, D, N, BH, kTile)) {
+      !host::make_map_cached(&mdk, dK, D, N, BH, kTile) || !host::make_map_cached(&mdv, dV, D, N, BH, kTile)) {
     snprintf(host::g_last_error, sizeof(host::g_last_error), "cuTensorMapEncodeTiled failed");
     return FA_ERR_CUDA;
   }
   const long long rows_pad = static_cast<long long>(BH) * prm.n_pad;
   bwd_rowdot_kernel<D><<<static_cast<unsigned>((rows_pad + 7) / 8), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), LSE, lse2, dd, N,
-      prm.n_pad, rows_pad);
+      static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), LSE, lse2, dd, prm.dq_acc,
+      N, prm.n_pad, rows_pad);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return host::cuda_fail(e, "bwd rowdot launch");
   const unsigned grid = static_cast<unsigned>(static_cast<long long>(BH) * prm.n_tiles);
   const int slot = (D == 128 ? 4 : 0) + (CAUSAL ? 2 : 0);
   fa_status r = set_smem(bwd_dkdv_kernel<D, CAUSAL>, DkdvCfg<D>::kSmemBytes, slot);
   if (r != FA_OK) return r;
-  r = set_smem(bwd_dq_kernel<D, CAUSAL>, DqCfg<D>::kSmemBytes, slot + 1);
-  if (r != FA_OK) return r;
   bwd_dkdv_kernel<D, CAUSAL><<<grid, kThreads, DkdvCfg<D>::kSmemBytes, st>>>(mq, mk, mv, mdo, mdk, mdv, prm);
   e = cudaGetLastError();
   if (e != cudaSuccess) return host::cuda_fail(e, "bwd dkdv launch");
-  bwd_dq_kernel<D, CAUSAL><<<grid, kThreads, DqCfg<D>::kSmemBytes, st>>>(mq, mk, mv, mdo, mdq, prm);
+  const long long rows = static_cast<long long>(BH) * N;
+  bwd_dq_convert_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
+      prm.dq_acc, static_cast<__nv_bfloat16*>(dQ), prm.scale, N, prm.n_pad, rows);
   e = cudaGetLastError();
-  if (e != cudaSuccess) return host::cuda_fail(e, "bwd dq launch");
+  if (e != cudaSuccess) return host::cuda_fail(e, "bwd dq convert launch");
   return FA_OK;
 }
 
@@ -843,9 +759,11 @@ int fa_bwd_trace_set(void* device_buffer) {
 
 size_t fa_bwd_workspace_bytes(int B, int H, int N) {
   if (B < 1 || H < 1 || N < 1) return 0;
-  // LSE * log2(e) and D = rowsum(dO * O), fp32, each [B][H][N rounded up to 128]
+  // LSE * log2(e) and D = rowsum(dO * O), fp32, each [B][H][N rounded up to
+  // 128]; then the fp32 dQ accumulator [B][H][N rounded up][d], sized for
+  // the largest head dimension (128)
   const size_t n_pad = (static_cast<size_t>(N) + fa::bwd::kTile - 1) / fa::bwd::kTile * fa::bwd::kTile;
-  return 2 * static_cast<size_t>(B) * H * n_pad * 4;
+  return (2 + 128) * static_cast<size_t>(B) * H * n_pad * 4;
 }
 
 fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
@@ -889,6 +807,7 @@ fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, con
   float* dd = lse2 + static_cast<size_t>(BH) * prm.n_pad;
   prm.lse2 = lse2;
   prm.dd = dd;
+  prm.dq_acc = dd + static_cast<size_t>(BH) * prm.n_pad;  // 1024-byte aligned: n_pad is a multiple of 128
   {
     // keep the Q, dO, K, V of one group of heads (8*N*d bytes per head) within ~48 MB of L2
     const long long per_head = 8ll * N * d;

@@ -325,11 +325,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 // tcgen05 MMA
 // ---------------------------------------------------------------------------
 // Instruction descriptor of kind::f16 with bf16 A and B and an fp32
-// accumulator.  b_mn_major: B stored with N contiguous (transpose bit).
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, bool b_mn_major) {
+// accumulator.  b_mn_major: B stored with N contiguous, a_mn_major: A stored
+// with M contiguous (the transpose bits).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, bool b_mn_major,
+                                                      bool a_mn_major = false) {
   return (1u << 4)                          // D format: f32
          | (1u << 7)                        // A format: bf16
          | (1u << 10)                       // B format: bf16
+         | ((a_mn_major ? 1u : 0u) << 15)   // A major
          | ((b_mn_major ? 1u : 0u) << 16)   // B major
          | ((N >> 3) << 17)                 // N / 8
          | ((M >> 4) << 24);                // M / 16

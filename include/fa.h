@@ -132,20 +132,25 @@ int fa_fwd_splitkv_default_splits(int B, int H, int N, int d, int causal);
  *   dQ, dK, dV      device, bf16 [B][H][N][d], written.
  *   workspace       device, 16-byte aligned, >= fa_bwd_workspace_bytes(B, H,
  *                   N) bytes, overwritten: LSE * log2(e) and D, each fp32
- *                   [B][H][N rounded up to 128].
+ *                   [B][H][N rounded up to 128], then the fp32 accumulator
+ *                   of dS K, [B][H][N rounded up to 128][d].
  *   B, H, N, d, scale, causal, stream: as for fa_fwd.
  * The outputs and the workspace must not overlap the inputs or each other.
- * Three kernels are enqueued on `stream`.  Errors as fa_fwd, plus
- * FA_ERR_WORKSPACE for a short workspace; device-side give-ups are reported
- * by fa_get_device_status().
+ * Three kernels are enqueued on `stream`: the row dots (and the accumulator
+ * cleared), dK and dV with every key tile's share of dQ added into the
+ * accumulator (fp32 reductions at L2, so dQ's rounding depends on the order
+ * in which they land: results may differ from run to run in the last bits),
+ * and dQ converted to bf16.  Errors as fa_fwd, plus FA_ERR_WORKSPACE for a
+ * short workspace; device-side give-ups are reported by
+ * fa_get_device_status().
  */
 fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                  const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
                  size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
                  void* stream);
 
-/* Bytes of workspace fa_bwd needs: 8 * B * H * (N rounded up to 128); 0 for
- * invalid arguments. */
+/* Bytes of workspace fa_bwd needs: (2 + 128) * 4 * B * H * (N rounded up to
+ * 128), enough for either head dimension; 0 for invalid arguments. */
 size_t fa_bwd_workspace_bytes(int B, int H, int N);
 
 /* Size of the workspace built into the library for fa_fwd_splitkv_noalloc. */

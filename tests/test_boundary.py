@@ -165,8 +165,9 @@ def test_bwd_argument_checks(lib):
     lib.fa_bwd.restype = ci
     lib.fa_bwd_workspace_bytes.argtypes = [ci, ci, ci]
     lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
-    assert lib.fa_bwd_workspace_bytes(2, 3, 100) == 2 * 2 * 3 * 128 * 4
-    assert lib.fa_bwd_workspace_bytes(1, 1, 129) == 2 * 256 * 4
+    # LSE*log2(e) and D per padded row, then the fp32 dQ accumulator (d <= 128)
+    assert lib.fa_bwd_workspace_bytes(2, 3, 100) == (2 + 128) * 2 * 3 * 128 * 4
+    assert lib.fa_bwd_workspace_bytes(1, 1, 129) == (2 + 128) * 256 * 4
     base = [A + k * 64 * MB for k in range(10)]  # Q K V O dO LSE dQ dK dV ws
 
     def bwd(args=None, ws_bytes=1 << 20, N=128, d=64):
