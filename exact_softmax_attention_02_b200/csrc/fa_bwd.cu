@@ -191,10 +191,12 @@ __device__ __forceinline__ void ds_16(const float (&p)[16], const uint32_t (&dp)
 // DS_SMEM: dS also goes to shared memory as the A operand of dQ_i = dS K:
 // [keys][queries] (query-contiguous, two 64-query chunks of 128-byte rows in
 // the 128-byte swizzle), row r = the thread's key; ds_row points at row r of
-// the first chunk.
-template <bool WRITE_P, bool MASK, bool DS_SMEM, typename Col, typename Allowed, typename Wait>
+// the first chunk.  each_quarter(q) runs at the start of quarter q (other
+// work to interleave with the quarters).
+template <bool WRITE_P, bool MASK, bool DS_SMEM, typename Col, typename Allowed, typename Wait,
+          typename Each>
 __device__ __forceinline__ bool p_ds_tile(uint32_t tS, uint32_t tDP, int h, float sl2, Col col,
-                                          Allowed allowed, uint64_t* ready, Wait dp_ready,
+                                          Allowed allowed, uint64_t* ready, Wait dp_ready, Each each_quarter,
                                           uint8_t* ds_row = nullptr, int r = 0) {
   uint32_t s[2][16], dp[16];
   tmem_ld16(tS + h * 16, s[0]);
@@ -203,6 +205,7 @@ __device__ __forceinline__ bool p_ds_tile(uint32_t tS, uint32_t tDP, int h, floa
   for (int q = 0; q < 4; ++q) {
     const int c0 = q * kQuarter + h * 16;
     if (q < 3) tmem_ld16(tS + c0 + kQuarter, s[(q + 1) & 1]);
+    each_quarter(q);
     float pv[16];
     p_16<MASK>(s[q & 1], c0, sl2, col, allowed, pv);
     if (q == 0) {
@@ -548,6 +551,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* box = sDs + e * C::kBoxBytes;  // this warp's transposition box
     const float sl2 = p.scale_log2;
     const bool tr = lane == 0 && wq == 0;
+    // A tile's share of dQ is added into the fp32 accumulator while the next
+    // tile is formed: 3/16 of it in each quarter and the last quarter of it
+    // while the dQ product of that tile is in the tensor core, so that the
+    // reductions reach L2 as a steady stream under the arithmetic instead of
+    // a burst the warps would stall on.  pend holds it transposed (see
+    // below); pend_base is its accumulator rows, null when nothing is
+    // pending.
+    constexpr int kRounds = D / 64;     // 32-column groups of this thread's half of a row
+    constexpr int kReds = kRounds * 8;  // reduction instructions per tile and thread
+    constexpr int kPerQuarter = kReds * 3 / 16;
+    float4 pend[kReds];
+    float* pend_base = nullptr;
+    auto flush = [&](int from, int to) {
+      if (pend_base == nullptr) return;
+#pragma unroll
+      for (int k = 0; k < kReds; ++k) {
+        if (k < from || k >= to) continue;
+        const int row = (k & 7) * 4 + (lane >> 3), g = lane & 7;
+        red_add_v4(pend_base + static_cast<size_t>(row) * D + (k >> 3) * 32 + g * 4, pend[k]);
+      }
+    };
     bool ok = true;
     for (int it = 0; it < n_iter && ok; ++it) {
       const int s = it % S;
@@ -577,16 +601,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (the previous tile's transposition is over: every warp passed the
       // barrier that ends it)
       uint8_t* ds_row = sDs + r * 128;
-      ok = diag ? p_ds_tile<true, true, true>(tS, tDP, h, sl2, col, allowed, ds_ready, dp_ready, ds_row, r)
-                : p_ds_tile<true, false, true>(tS, tDP, h, sl2, col, allowed, ds_ready, dp_ready, ds_row, r);
+      auto each_quarter = [&](int q) { flush(q * kPerQuarter, (q + 1) * kPerQuarter); };
+      ok = diag ? p_ds_tile<true, true, true>(tS, tDP, h, sl2, col, allowed, ds_ready, dp_ready, each_quarter,
+                                              ds_row, r)
+                : p_ds_tile<true, false, true>(tS, tDP, h, sl2, col, allowed, ds_ready, dp_ready, each_quarter,
+                                               ds_row, r);
       if (tr) BWD_TRACE(0, 1 + h, it, 1);
       if (!ok) break;
+      flush(4 * kPerQuarter, kReds);
       // dQ_i: this thread's query row r, columns [h d/2, (h+1) d/2), 32 at a time
       ok = __all_sync(0xffffffffu,
                       mbar_wait(dq_full, static_cast<uint32_t>(it) & 1u, abort_flag, status, tmo, kSiteDq));
       if (!ok) break;
       tc_fence_after();
-      constexpr int kRounds = D / 64;
       uint32_t o[kRounds][32];
 #pragma unroll
       for (int rd = 0; rd < kRounds; ++rd) tmem_ld32(tDQ + h * (D / 2) + rd * 32, o[rd]);
@@ -594,14 +621,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_drained);
-      // Added into the fp32 accumulator 32 columns at a time through this
-      // warp's box (the dQ_i product has finished, so dS is no longer read
-      // and its buffer holds the boxes): each lane writes its row (128 bytes,
-      // 16-byte granules rotated by the row to spread the banks), then the
-      // warp reads the box back four rows per instruction, eight lanes per
-      // row, so that every reduction instruction covers four whole 128-byte
-      // lines of the accumulator.
-      float* acc_base = p.dq_acc + (static_cast<size_t>(bh) * p.n_pad + i * kTile + wq * 32) * D + h * (D / 2);
+      // Transposed 32 columns at a time through this warp's box (the dQ_i
+      // product has finished, so dS is no longer read and its buffer holds
+      // the boxes): each lane writes its row (128 bytes, 16-byte granules
+      // rotated by the row to spread the banks), then the warp reads the box
+      // back four rows per instruction, eight lanes per row, so that every
+      // reduction instruction covers four whole 128-byte lines of the
+      // accumulator.
 #pragma unroll
       for (int rd = 0; rd < kRounds; ++rd) {
 #pragma unroll
@@ -612,16 +638,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k4 = 0; k4 < 8; ++k4) {
           const int row = k4 * 4 + (lane >> 3), g = lane & 7;
-          const float4 v = *reinterpret_cast<const float4*>(box + row * 128 + ((g ^ (row & 7)) * 16));
-          red_add_v4(acc_base + static_cast<size_t>(row) * D + rd * 32 + g * 4, v);
+          pend[rd * 8 + k4] = *reinterpret_cast<const float4*>(box + row * 128 + ((g ^ (row & 7)) * 16));
         }
         __syncwarp();  // the box is read before the next round overwrites it
       }
+      pend_base = p.dq_acc + (static_cast<size_t>(bh) * p.n_pad + i * kTile + wq * 32) * D + h * (D / 2);
       // the next tile's dS goes into the same buffer: every warp must have
       // read its boxes back first
       named_bar_sync(3, kElemThreads);
       if (tr) BWD_TRACE(0, 1 + h, it, 2);
     }
+    if (ok) flush(0, kReds);  // the last tile's share
     if (ok) ok = mbar_wait(acc_done, 0, abort_flag, status, tmo, kSiteO);
     const bool failed = named_bar_or(2, kElemThreads, !ok);
     if (!failed && n_iter > 0) {
