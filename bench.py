@@ -398,7 +398,7 @@ def measure_config(name: str, path: str, dev, steps: int = 20, warmup: int = 5):
            "ms_per_step": 1e3 * mean_s,
            "ms_min": ms[0], "ms_median": ms[len(ms) // 2], "steps": steps, "warmup": warmup,
            "flops_per_step": flops, "clocks": sampler.summary(),
-           "kernel": ("bwd_rowdot + bwd_dkdv_kernel + bwd_dq_kernel" if path == "backward"
+           "kernel": ("bwd_rowdot + bwd_dkdv_kernel + bwd_dq_convert" if path == "backward"
                       else f"fa_fwd_kernel<{w.d},{str(w.causal).lower()}>"),
            "launches": steps * (3 if path == "backward" else 1)}
     if path == "backward":
@@ -574,7 +574,7 @@ def run_ours(args, w):
                 "kernel_source_sha256": kernel_source_hash()}
     if bwd is not None:
         # one step = rowdot + dK/dV + dQ kernels, timed together
-        roofline.update(kernel="bwd_rowdot + bwd_dkdv_kernel + bwd_dq_kernel", traffic=None,
+        roofline.update(kernel="bwd_rowdot + bwd_dkdv_kernel + bwd_dq_convert", traffic=None,
                         flops_convention="2.5 x forward (five N^2 d products)")
     if args.path == "standard":
         # the comparator's dominant kernel is the HBM-bound row softmax:

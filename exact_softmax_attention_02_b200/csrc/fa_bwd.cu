@@ -344,8 +344,8 @@ struct DkdvCfg {
 //   and dK += dS^T Q_i run on one quarter while the next is being formed;
 //   they also write dS to shared memory, and dQ_i = dS K (the tile's share of
 //   dQ for query tile i) is then formed in TMEM, read out by the elementwise
-//   warps and added into the fp32 dQ accumulator in global memory by TMA
-//   reduce-adds.  So every product of the gradient is computed once: no
+//   warps and added into the fp32 dQ accumulator in global memory by
+//   reductions at L2.  So every product of the gradient is computed once: no
 //   second pass recomputes S and dP for dQ.
 // tcgen05 MMAs of one thread run in issue order, so dP^T of tile i+1 may be
 // issued right after the products that read tile i's dS^T, and S^T of tile
