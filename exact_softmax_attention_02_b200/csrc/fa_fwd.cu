@@ -568,6 +568,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 FA_TRACE_MARK(0, trace_it + it, 3 * t + 1);
                 if (last) mma_commit(&o_full[t]);
               }
+              // the V stage is free once the second tile's PV has read it,
+              // ahead of that tile's next S product (+1.3% on causal N = 8192
+              // against releasing it with the K stage after that S)
+              if (t == 1) mma_commit(&kv_empty[sv]);
               if (!last && it + 1 >= u.first_it[t]) {
                 if (!q_ready[t]) {
                   if (!(ok = wait_q(t))) break;
@@ -581,7 +585,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
             if (!ok) break;
-            mma_commit(&kv_empty[sv]);
             if (!last) mma_commit(&kv_empty[sk]);
           }
           i = i0 + 2 * n_iter;
