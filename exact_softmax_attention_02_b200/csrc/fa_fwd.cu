@@ -76,17 +76,20 @@ constexpr int kSoftmaxWarp0 = 4;
 // Registers per thread after the split between warpgroup 0 (producer, MMA,
 // two idle warps) and the two softmax warpgroups, with 128 * control + 256 *
 // softmax = 384 * 168, the 64K register file at the launch's 168 per thread:
-// the smallest control share that compiles without spills (found with
-// -Xptxas -v), the rest to the softmax.
+// the smallest control share that compiles without spills in every
+// variant (found with -Xptxas -v), the rest to the softmax.
 template <int D, bool CAUSAL, bool SPLIT, bool SPARSE>
 __host__ __device__ constexpr uint32_t regs_control() {
-  return (D == 64 && CAUSAL && !SPLIT && !SPARSE) ? 152 : 136;
+  return 136;
 }
 template <int D, bool CAUSAL, bool SPLIT, bool SPARSE>
 __host__ __device__ constexpr uint32_t regs_softmax() {
   return (kThreads * 168 - 128 * regs_control<D, CAUSAL, SPLIT, SPARSE>()) / 256;
 }
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// a tile whose row sum of p (against the lagging reference maximum) stays
+// within 2^16 keeps the reference
+constexpr float kLazySum = 65536.0f;
 constexpr uint32_t kTmemCols = 512;
 // wait sites reported in the device status word (bit 8 + site)
 enum : uint32_t {
@@ -690,63 +693,116 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (kbase + q * 32 + cc > lim) sr[q][cc] = __float_as_uint(-INFINITY);
           }
           // row maximum of the raw scores (scale > 0 keeps the argmax): BN/16
-          // independent chains of three-input maxima
-          constexpr int kChains = BN / 16;
-          float mx[kChains];
+          // independent chains of three-input maxima; log2 units of scaled scores
+          auto tile_max = [&]() {
+            constexpr int kChains = BN / 16;
+            float mx[kChains];
   #pragma unroll
-          for (int kx = 0; kx < kChains; ++kx) mx[kx] = __uint_as_float(sr[kx >> 1][(kx & 1) * 16]);
+            for (int kx = 0; kx < kChains; ++kx) mx[kx] = __uint_as_float(sr[kx >> 1][(kx & 1) * 16]);
   #pragma unroll
-          for (int kx = 0; kx < kChains; ++kx) {
-            const uint32_t* v = &sr[kx >> 1][(kx & 1) * 16];
+            for (int kx = 0; kx < kChains; ++kx) {
+              const uint32_t* v = &sr[kx >> 1][(kx & 1) * 16];
   #pragma unroll
-            for (int cc = 1; cc < 15; cc += 2)
-              mx[kx] = fmax3(mx[kx], __uint_as_float(v[cc]), __uint_as_float(v[cc + 1]));
-            mx[kx] = fmaxf(mx[kx], __uint_as_float(v[15]));
-          }
-          float m_all;
-          if constexpr (kChains == 8)
-            m_all = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-          else
-            m_all = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]);
-          const float m_tile = m_all * sl2;
-          if (tr) FA_TRACE_MARK(1 + t, trace_it + it, 2);
-          // raise the reference maximum only when this tile exceeds it by > 2^8
-          const bool raise = m_tile > m_ref + kRescaleThreshold;
+              for (int cc = 1; cc < 15; cc += 2)
+                mx[kx] = fmax3(mx[kx], __uint_as_float(v[cc]), __uint_as_float(v[cc + 1]));
+              mx[kx] = fmaxf(mx[kx], __uint_as_float(v[15]));
+            }
+            float m_all;
+            if constexpr (kChains == 8)
+              m_all = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+            else
+              m_all = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]);
+            return m_all * sl2;
+          };
+          const float2 sl2v = make_float2(sl2, sl2);
+          float2 ps2[kQ32];
+          // p = 2^(s * scale * log2 e - m_ref), written as bf16 pairs over the
+          // first BN/2 columns of S_t, 64 keys at a time, and published whole
+          // on p_full[t]; ps2 gets the row sums of the fp32 p.  The keys are
+          // taken from the top down, so that the scores of keys [0, BN/2),
+          // whose columns the P stores overwrite, are the last ones read:
+          // they stay in registers for a redo (below), while those of keys
+          // [BN/2, BN) remain in TMEM.
+          auto exponentials = [&]() {
+            const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+            const float2 nm2 = make_float2(neg_m, neg_m);
+  #pragma unroll
+            for (int h = BN / 64 - 1; h >= 0; --h) {
+              // keys [64h, 64h + 64) -> 32 columns of bf16 pairs at column 32h
+              uint32_t pk[32];
+  #pragma unroll
+              for (int qq = 1; qq >= 0; --qq) {
+                const int q = 2 * h + qq;
+                ps2[q] = make_float2(0.f, 0.f);
+  #pragma unroll
+                for (int cc = 0; cc < 32; cc += 2) {
+                  const float2 x = ffma2(make_float2(__uint_as_float(sr[q][cc]), __uint_as_float(sr[q][cc + 1])),
+                                         sl2v, nm2);
+                  float2 pv;
+                  pv.x = ex2_approx(x.x);
+                  pv.y = ex2_approx(x.y);
+                  ps2[q] = fadd2(ps2[q], pv);
+                  pk[qq * 16 + (cc >> 1)] = pack_bf16x2(pv.x, pv.y);
+                }
+              }
+              tmem_st32(tS + h * 32, pk);
+              if (tr && h == BN / 64 - 1) FA_TRACE_MARK(1 + t, trace_it + it, 3);
+            }
+          };
+          auto row_sum = [&]() {
+            float2 psum;
+            if constexpr (kQ32 == 4)
+              psum = fadd2(fadd2(ps2[0], ps2[1]), fadd2(ps2[2], ps2[3]));
+            else
+              psum = fadd2(ps2[0], ps2[1]);
+            return psum.x + psum.y;
+          };
+          // The reference maximum m_ref lags the row maximum: it is raised
+          // only when a tile's scores exceed it by more than
+          // kRescaleThreshold.  In a row block's first tile the maximum is
+          // taken before the exponentials.  After that it is not: the
+          // exponentials run against m_ref, and a row sum of at most kLazySum
+          // (2^16) bounds every p of the tile by it, so m_ref may stay (fp32
+          // and bf16 hold such p with their full relative precision).  Only a warp with a larger sum (or a row still
+          // without a reference) takes the maximum and redoes the tile.
           float alpha = 1.f;
-          if (raise) {
-            alpha = ex2_approx(m_ref - m_tile);  // 0 while m_ref is -inf
-            m_ref = m_tile;
+          bool raise = false;
+          auto raise_ref = [&]() {
+            const float m_tile = tile_max();
+            raise = m_tile > m_ref + kRescaleThreshold;
+            if (raise) {
+              alpha = ex2_approx(m_ref - m_tile);  // 0 while m_ref is -inf
+              m_ref = m_tile;
+            }
+          };
+          if (li == 0) {
+            raise_ref();
+            if (tr) FA_TRACE_MARK(1 + t, trace_it + it, 2);
+            exponentials();
+          } else {
+            if (tr) FA_TRACE_MARK(1 + t, trace_it + it, 2);
+            exponentials();
+            const float sum = row_sum();
+            if (__any_sync(0xffffffffu, !(sum <= kLazySum) || m_ref == -INFINITY)) {
+              // the scores of keys [BN/2, BN) back from TMEM (their columns
+              // hold no P)
+  #pragma unroll
+              for (int q = kQ32 / 2; q < kQ32; ++q) tmem_ld32(tS + q * 32, sr[q]);
+              tmem_wait_ld();
+              if (masked) {
+                const int lim = bad ? -1 : key_limit;
+  #pragma unroll
+                for (int q = kQ32 / 2; q < kQ32; ++q)
+  #pragma unroll
+                  for (int cc = 0; cc < 32; ++cc)
+                    if (kbase + q * 32 + cc > lim) sr[q][cc] = __float_as_uint(-INFINITY);
+              }
+              raise_ref();
+              // (the stores of P are warp-wide: every lane writes its row again)
+              if (__any_sync(0xffffffffu, raise)) exponentials();
+            }
           }
           const bool rescale_o = li > 0 && __any_sync(0xffffffffu, raise);
-          const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-          const float2 sl2v = make_float2(sl2, sl2);
-          const float2 nm2 = make_float2(neg_m, neg_m);
-          float2 ps2[kQ32];
-          // p = 2^(s * scale * log2 e - m), written as bf16 pairs over the first
-          // BN/2 columns of S_t, 64 keys at a time, and published whole on
-          // p_full[t].
-  #pragma unroll
-          for (int h = 0; h < BN / 64; ++h) {
-            // keys [64h, 64h + 64) -> 32 columns of bf16 pairs at column 32h
-            uint32_t pk[32];
-  #pragma unroll
-            for (int qq = 0; qq < 2; ++qq) {
-              const int q = 2 * h + qq;
-              ps2[q] = make_float2(0.f, 0.f);
-  #pragma unroll
-              for (int cc = 0; cc < 32; cc += 2) {
-                const float2 x = ffma2(make_float2(__uint_as_float(sr[q][cc]), __uint_as_float(sr[q][cc + 1])),
-                                       sl2v, nm2);
-                float2 pv;
-                pv.x = ex2_approx(x.x);
-                pv.y = ex2_approx(x.y);
-                ps2[q] = fadd2(ps2[q], pv);
-                pk[qq * 16 + (cc >> 1)] = pack_bf16x2(pv.x, pv.y);
-              }
-            }
-            tmem_st32(tS + h * 32, pk);
-            if (tr && h == 0) FA_TRACE_MARK(1 + t, trace_it + it, 3);
-          }
           // the rescale waits until the scores have left the registers
           if (rescale_o) rescale_o_rows(tO, alpha);
           // every lane's stores have completed; one arrival per warp
@@ -755,12 +811,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&p_full[t]);
           if (lane == 0 && wq != 0) FA_TRACE_MARK(1 + t, trace_it + it, 4 + wq);
-          float2 psum;
-          if constexpr (kQ32 == 4)
-            psum = fadd2(fadd2(ps2[0], ps2[1]), fadd2(ps2[2], ps2[3]));
-          else
-            psum = fadd2(ps2[0], ps2[1]);
-          l_sum = l_sum * alpha + (psum.x + psum.y);
+          l_sum = l_sum * alpha + row_sum();
           if (tr) FA_TRACE_MARK(1 + t, trace_it + it, 4);
         }
         trace_it += n_iter;
