@@ -297,3 +297,31 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     assert fa.device_status() == 0  # status was cleared
     # the context is still usable and results are right again
     compare(q, k, v, True, every_row(1, 2, 512))
+
+
+# ---------------------------------------------------------------------------
+# the lagging reference maximum
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("j0", [5, 200])
+@pytest.mark.parametrize("jump", [12.0, 40.0, 200.0])
+def test_reference_maximum_raised_by_a_later_tile(d, causal, j0, jump):
+    """The key tiles are visited from the last one down. After a row block's first
+    tile, the kernel keeps its reference maximum unless a tile's row sum of
+    p = 2^(s - reference) exceeds 2^16. Key j0 sits in a tile visited after the first.
+    A feature that only it carries lifts its score about `jump` (natural-log units of
+    the scaled score) above the rest:
+    - at 12, p stays within 2^16 for most rows, and the reference is kept;
+    - at 40, the row sum exceeds 2^16, and the warp takes the maximum and redoes the
+      tile;
+    - at 200, p overflows to infinity before the redo.
+    Every row is checked against the oracle."""
+    B, H, N = 1, 2, 512
+    q, k, v = make_qkv(B, H, N, d, seed=11)
+    scale = 1.0 / math.sqrt(d)
+    q[..., 0] = 1.0
+    k[..., 0] = 0.0
+    k[:, :, j0, 0] = jump / scale
+    compare(q, k, v, causal, every_row(B, H, N), scale=scale)
