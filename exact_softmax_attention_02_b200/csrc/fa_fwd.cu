@@ -767,6 +767,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // without a reference) takes the maximum and redoes the tile.
           float alpha = 1.f;
           bool raise = false;
+          bool maxed = li == 0;  // the tile's maximum was taken (only then may a row raise)
           auto raise_ref = [&]() {
             const float m_tile = tile_max();
             raise = m_tile > m_ref + kRescaleThreshold;
@@ -784,6 +785,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             exponentials();
             const float sum = row_sum();
             if (__any_sync(0xffffffffu, !(sum <= kLazySum) || m_ref == -INFINITY)) {
+              maxed = true;
               // the scores of keys [BN/2, BN) back from TMEM (their columns
               // hold no P)
   #pragma unroll
@@ -802,7 +804,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (__any_sync(0xffffffffu, raise)) exponentials();
             }
           }
-          const bool rescale_o = li > 0 && __any_sync(0xffffffffu, raise);
+          // (no vote when no row could have raised: +0.7% on causal N = 8192)
+          const bool rescale_o = li > 0 && maxed && __any_sync(0xffffffffu, raise);
           // the rescale waits until the scores have left the registers
           if (rescale_o) rescale_o_rows(tO, alpha);
           // every lane's stores have completed; one arrival per warp
