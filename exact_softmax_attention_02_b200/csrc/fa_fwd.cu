@@ -547,7 +547,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int iv = i0 + 2 * it + 1, ik = i0 + 2 * it + 2;
             const int sv = iv % S, sk = ik % S;
             const bool last = it == n_iter - 1;
-            if (!(ok = wait_load(iv))) break;
+            // At d = 64 each V after the item's first is waited for earlier,
+            // between the previous key tile's PV and S products of query tile
+            // 1 (+1.7% there; -2.9% at d = 128, where that wait delays the S
+            // products of the longer PV/S blocks)
+            constexpr bool kEarlyV = D == 64;
+            if ((!kEarlyV || it == 0) && !(ok = wait_load(iv))) break;
             FA_TRACE_MARK(3, trace_it + it, 0);
             // the next K tile too, here rather than between a PV and an S
             // product: it has normally landed long before, but the wait itself
@@ -575,6 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               // ahead of that tile's next S product (+1.3% on causal N = 8192
               // against releasing it with the K stage after that S)
               if (t == 1) mma_commit(&kv_empty[sv]);
+              if (kEarlyV && t == 1 && !last && !(ok = wait_load(iv + 2))) break;
               if (!last && it + 1 >= u.first_it[t]) {
                 if (!q_ready[t]) {
                   if (!(ok = wait_q(t))) break;
