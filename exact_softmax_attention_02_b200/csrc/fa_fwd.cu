@@ -476,12 +476,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t skv = smem_addr(sKV);
       // The issuing thread is on the critical path between the softmax and
       // the next S (an MMA is accepted only about as fast as the tensor core
-      // retires the one before), so at d = 128 each operand's descriptor is
-      // built once per product and advanced by a constant per K-step (the
-      // start-address field counts 16-byte units and shared-memory addresses
-      // stay below 2^18, so adding the offset never carries out of it).
-      // Measured on B200: +2.6% at d = 128, -1.5% at d = 64 (kept off there).
-      constexpr bool kAdvanceDesc = D == 128;
+      // retires the one before), so each operand's descriptor is built once
+      // per product and advanced by a constant per K-step (the start-address
+      // field counts 16-byte units and shared-memory addresses stay below
+      // 2^18, so adding the offset never carries out of it).  Measured on
+      // B200: +2.6% at d = 128, +1.2% at d = 64.
       // S_t = Q_t K^T: A = Q_t (K-major), B = K stage (K-major); 16 columns of
       // d per instruction, 32 bytes apart inside each 128-byte swizzled row.
       auto issue_s = [&](int t, int s) {
@@ -491,9 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t aoff = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
           const uint32_t boff = (kk >> 2) * C::kKChunkBytes + (kk & 3) * 32;
-          const uint64_t ad = kAdvanceDesc ? a0 + (aoff >> 4) : sw128_desc(sq + t * QB + aoff, 16, 1024);
-          const uint64_t bd = kAdvanceDesc ? b0 + (boff >> 4) : sw128_desc(skv + s * SB + boff, 16, 1024);
-          mma_ss(tmem + t * BN, ad, bd, idS, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + t * BN, a0 + (aoff >> 4), b0 + (boff >> 4), idS, kk > 0 ? 1u : 0u);
         }
       };
       // O_t (+)= P_t V: A = P_t in TMEM (8 columns per 16 keys), B = V stage
@@ -502,8 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t v0 = sw128_desc(skv + s * SB, C::kVChunkBytes, 1024);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bd = kAdvanceDesc ? v0 + static_cast<uint32_t>(kk * (2048 >> 4))
-                                           : sw128_desc(skv + s * SB + kk * 2048, C::kVChunkBytes, 1024);
+          const uint64_t bd = v0 + static_cast<uint32_t>(kk * (2048 >> 4));
           const uint32_t acc = (accumulate || kk > 0) ? 1u : 0u;
           mma_ts(tmem + C::kColO + t * D, tmem + t * BN + kk * 8, bd, idO, acc);
         }
