@@ -765,8 +765,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           // taken before the exponentials.  After that it is not: the
           // exponentials run against m_ref, and a row sum of at most kLazySum
           // (2^16) bounds every p of the tile by it, so m_ref may stay (fp32
-          // and bf16 hold such p with their full relative precision).  Only a warp with a larger sum (or a row still
-          // without a reference) takes the maximum and redoes the tile.
+          // and bf16 hold such p with their full relative precision).  Only
+          // a warp with a larger sum (or a row still without a reference)
+          // takes the maximum and redoes the tile.
           float alpha = 1.f;
           bool raise = false;
           bool maxed = li == 0;  // the tile's maximum was taken (only then may a row raise)
