@@ -306,15 +306,16 @@ def test_bounded_wait_reports_timeout_and_context_survives():
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("j0", [5, 200])
-@pytest.mark.parametrize("jump", [12.0, 40.0, 200.0])
+@pytest.mark.parametrize("jump", [12.0, 20.0, 40.0, 200.0])
 def test_reference_maximum_raised_by_a_later_tile(d, causal, j0, jump):
     """The key tiles are visited from the last one down. After a row block's first
     tile, the kernel keeps its reference maximum unless a tile's row sum of
-    p = 2^(s - reference) exceeds 2^16. Key j0 sits in a tile visited after the first.
+    p = 2^(s - reference) exceeds 2^30. Key j0 sits in a tile visited after the first.
     A feature that only it carries lifts its score about `jump` (natural-log units of
     the scaled score) above the rest:
-    - at 12, p stays within 2^16 for most rows, and the reference is kept;
-    - at 40, the row sum exceeds 2^16, and the warp takes the maximum and redoes the
+    - at 12, p stays far within 2^30, and the reference is kept;
+    - at 20, p reaches ~2^24: the reference is kept with a lag of ~24 (log2 units);
+    - at 40, the row sum exceeds 2^30, and the warp takes the maximum and redoes the
       tile;
     - at 200, p overflows to infinity before the redo.
     Every row is checked against the oracle."""
